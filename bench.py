@@ -1,0 +1,425 @@
+"""Benchmark: block-causal chunk attention over a Wan2.1-1.3B-shaped 5-step wavefront.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {wf,reference}] [--config 2]
+
+One step is one pass of the whole hot path over one layer of the wavefront: wf_kv_append of the
+five active chunks' K/V into their pages (the two clean context chunks are appended once, before
+timing) and one wf_attn_forward over all chunks.  Inputs are seeded synthetic tensors of the
+workload's shapes, resident in HBM before the timed region (q 72 MB, K/V 144 MB appended per step,
+201 MB of K/V pages read, 72 MB written: far larger than the 126 MB L2).
+
+Printed (rank 0, one JSON line): throughput in TFLOP/s of algorithmic attention work
+(4 * D * H * sum over query rows of visible keys; masked pairs, exp and rescaling not counted),
+with tokens/s, the roofline of the attention kernel, an end-to-end figure through the C ABI with
+host buffers, the CPU oracle as a baseline, and the SM clocks seen during the timed region.
+
+With --gpus N > 1 (launched by torch.distributed.run) every rank runs an independent replica of
+the same workload: the path has no exchange step, so there is no data-path collective; a barrier
+and a max-reduction of the device times are the only collectives.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_causal_streaming_b200.workloads import CONFIGS, Workload, make_inputs  # noqa: E402
+
+METRIC = "block-causal chunk-attention TFLOP/s and % of B200 bf16 peak; tokens/s"
+UNIT = "TFLOP/s"
+KERNEL_SOURCES = ["block_causal_streaming_b200/csrc/attn_kernel.cuh",
+                  "block_causal_streaming_b200/csrc/sm100.cuh"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------------------ accounting
+def attention_flops(wl: Workload) -> int:
+    """4 * D * H * sum over query rows of the number of keys that row may see."""
+    off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
+    visible = sum((off[c + 1] - off[c]) * off[c + 1] for c in range(nctx, wl.num_chunks))
+    return 4 * wl.head_dim * wl.heads * visible
+
+
+def rows_flops(wl: Workload, rows, heads_per_row: int) -> int:
+    off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
+    t_ctx = off[nctx]
+    total = 0
+    for r in rows:
+        t = t_ctx + r
+        c = next(i for i in range(wl.num_chunks) if off[i] <= t < off[i + 1])
+        total += off[c + 1]
+    return 4 * wl.head_dim * heads_per_row * total
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic():
+    """DRAM bytes per attention launch from a committed ncu capture, if it matches this kernel."""
+    path = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_hash") != kernel_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------ distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend,
+                                             timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        if device is not None and torch.distributed.get_backend() == "nccl":
+            torch.distributed.barrier(device_ids=[device.index])
+        else:
+            torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64,
+                     device=device if torch.distributed.get_backend() == "nccl" else "cpu")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(units_per_rank: float, world: int, seconds_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / seconds_max
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock, power and throttle reasons while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.reader.join(timeout=2)
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, flag in enumerate(r[3])
+                          if flag.lower() == "active"})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def oracle_sample(wl: Workload, inp, target_s: float, seed: int = 0):
+    """Time the oracle on a bounded sample of query rows (all heads); returns (TFLOP/s, info)."""
+    import oracle  # CPU-baseline leg only
+    rng = np.random.default_rng(seed)
+    q32 = inp.q.float().numpy()
+    k32 = inp.k.float().numpy()
+    v32 = inp.v.float().numpy()
+    scale = 1.0 / np.sqrt(wl.head_dim)
+    H = wl.heads
+
+    def run(rows):
+        rr = np.repeat(np.asarray(rows, dtype=np.int32), H)
+        hh = np.tile(np.arange(H, dtype=np.int32), len(rows))
+        t0 = time.perf_counter()
+        oracle.attention_rows(q32, k32, v32, wl.chunk_offsets, wl.num_ctx_chunks, scale, rr, hh)
+        return time.perf_counter() - t0
+
+    probe = sorted(rng.choice(wl.t_q, size=4, replace=False).tolist())
+    t_probe = run(probe)
+    per_row = t_probe / len(probe)
+    n = int(max(4, min(wl.t_q, target_s / max(per_row, 1e-6))))
+    rows = sorted(rng.choice(wl.t_q, size=n, replace=False).tolist())
+    dt = run(rows)
+    fl = rows_flops(wl, rows, H)
+    info = {"rows": n, "heads": H, "seconds": round(dt, 3), "flop": fl}
+    return fl / dt / 1e12, info
+
+
+# ------------------------------------------------------------------------------ GPU arm
+def gpu_arm(args, world, rank, local):
+    import block_causal_streaming_b200 as wf
+    from block_causal_streaming_b200.layer import PagedPool, WavefrontLayer
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    wl = CONFIGS[args.config]
+    inp = make_inputs(wl)
+    H, D = wl.heads, wl.head_dim
+    off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
+    scale = 1.0 / np.sqrt(D)
+    flop = attention_flops(wl)
+
+    pool = PagedPool(wl.num_pages, wl.page_size, H, D, dev)
+    pt = inp.page_table.to(dev).reshape(1, -1).contiguous()
+    layer = WavefrontLayer(pool, pt, 0, off, wl.chunk_stage, nctx)
+    q = inp.q.to(dev)
+    k = inp.k.to(dev)
+    v = inp.v.to(dev)
+    out = torch.empty_like(q)
+    active = list(range(nctx, wl.num_chunks))
+    layer.append_range(k, v, range(nctx))            # clean context: published once
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = len(active) + 1
+
+    def step(ev_pair=None):
+        layer.append_range(k, v, active)
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        layer.forward(q, out, scale=scale)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    rc = wf.check_status()
+    if rc != wf.WF_OK:
+        raise RuntimeError(f"device status after warm-up: {wf.strerror(rc)}")
+
+    # ---- timed region: K steps, device time by CUDA events on the launching stream
+    attn_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(attn_events[i])
+        t_stop.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+    elapsed = t_start.elapsed_time(t_stop) / 1e3
+    attn_ms = [a.elapsed_time(b) for a, b in attn_events]
+    elapsed_max = max_over_ranks(elapsed, world, dev)
+    rc = wf.check_status()
+    if rc != wf.WF_OK:
+        raise RuntimeError(f"device status after timing: {wf.strerror(rc)}")
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the region
+    q_h = inp.q.pin_memory()
+    act_rows = slice(off[nctx], off[-1])
+    k_h = inp.k[act_rows].contiguous().pin_memory()
+    v_h = inp.v[act_rows].contiguous().pin_memory()
+    out_h = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    k_act = torch.empty(k_h.shape, dtype=torch.bfloat16, device=dev)
+    v_act = torch.empty(v_h.shape, dtype=torch.bfloat16, device=dev)
+    q_in = torch.empty_like(q)
+    h2d = q_h.numel() * 2 + k_h.numel() * 2 + v_h.numel() * 2
+    d2h = out_h.numel() * 2
+
+    def e2e_step():
+        q_in.copy_(q_h, non_blocking=True)
+        k_act.copy_(k_h, non_blocking=True)
+        v_act.copy_(v_h, non_blocking=True)
+        base = off[nctx]
+        for c in active:
+            a, b = off[c] - base, off[c + 1] - base
+            layer.append(c, k_act[a:b], v_act[a:b])
+        layer.forward(q_in, out, scale=scale)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        e2e_step()
+    e_steps = max(3, min(args.steps, 10))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+    rc = wf.check_status()
+    if rc != wf.WF_OK:
+        raise RuntimeError(f"device status after end-to-end run: {wf.strerror(rc)}")
+
+    peaks, peak_src = load_peaks()
+    step_s = elapsed_max / args.steps
+    value = aggregate(flop, world, step_s) / 1e12
+    attn_avg_s = statistics.mean(attn_ms) / 1e3
+    achieved = flop / attn_avg_s / 1e12
+    peak = float(peaks["bf16_tflops"])
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_s * 1e3, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)*0.5 bf16)",
+        "config": {"workload": wl.name, "heads": H, "head_dim": D, "t_q": wl.t_q,
+                   "t_kv": wl.t_kv, "chunks": f"{nctx} ctx + {len(active)} active x 4680",
+                   "page_size": wl.page_size, "step": "append 5 active chunks + attention",
+                   "l2": "inputs larger than L2 (~490 MB touched per step vs 126 MB L2)",
+                   "parallelism": f"replicas x{world}"},
+        "tokens_per_s": round(world * wl.t_q / step_s, 1),
+        "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "roofline": {"bound": "tensor", "kernel": "wf_attn_fwd_kernel<128>",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": load_traffic(),
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "attn_ms_avg": round(attn_avg_s * 1e3, 4),
+                     "attn_ms_p50": round(statistics.median(attn_ms), 4)},
+        "e2e": {"value": round(aggregate(flop, world, e_elapsed / e_steps) / 1e12, 2),
+                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        tflops, info = oracle_sample(wl, inp, target_s=args.cpu_seconds)
+        res["cpu_baseline"] = {"value": round(tflops, 6), "unit": UNIT,
+                               "cores": os.cpu_count(), "kind": "oracle",
+                               "sample": f"{info['rows']} random query rows x {info['heads']} "
+                                         f"heads of the same workload, {info['seconds']} s"}
+    if world > 1:
+        torch.distributed.barrier(device_ids=[dev.index])
+        torch.distributed.destroy_process_group()
+    return res
+
+
+# ------------------------------------------------------------------------------ reference arm
+def reference_arm(args, world, rank):
+    """The oracle as it stands, on the host cores, on bounded samples of the same workload."""
+    if rank != 0:
+        return None
+    wl = CONFIGS[args.config]
+    inp = make_inputs(wl)
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    for i in range(args.warmup):
+        oracle_sample(wl, inp, target_s=min(per_step, 1.0), seed=1000 + i)
+    vals, secs, rows = [], 0.0, 0
+    for i in range(args.steps):
+        v, info = oracle_sample(wl, inp, target_s=per_step, seed=i)
+        vals.append(v)
+        secs += info["seconds"]
+        rows += info["rows"]
+    value = statistics.mean(vals)
+    sample = f"{args.steps} steps, each a random sample of query rows x {wl.heads} heads " \
+             f"({rows} rows, {secs:.1f} s total)"
+    return {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / args.steps, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1)*0.5 bf16)", "impl": "reference",
+        "config": {"workload": wl.name, "heads": wl.heads, "head_dim": wl.head_dim,
+                   "t_q": wl.t_q, "t_kv": wl.t_kv, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": os.cpu_count(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["wf", "reference"], default="wf")
+    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 5])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if world != args.gpus and world != 1:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        res = reference_arm(args, world, rank)
+    else:
+        res = gpu_arm(args, world, rank, local)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

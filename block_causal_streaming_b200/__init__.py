@@ -1,0 +1,25 @@
+"""B200-native (sm_100a) block-causal chunk attention for Wave Forcing wavefronts.
+
+The product is the C-ABI library ``libwf_b200.so`` (declared in ``include/wf.h``):
+
+* ``wf_kv_append``    -- publish one chunk's layer-wise K/V into fixed-size pages;
+* ``wf_attn_forward`` -- one block-causal attention over every chunk of the wavefront, one launch.
+
+This package is its thin Python binding (ctypes, argument marshalling only), a small helper that
+owns the paged pools of one layer (:mod:`.layer`) and the seeded synthetic workloads
+(:mod:`.workloads`).  The binding is loaded on first use of any of its names and fails loudly if
+the library has not been built; there is no CPU fallback.
+"""
+_ABI_NAMES = (
+    "WF_OK", "WF_ERR_INVALID_ARG", "WF_ERR_SHAPE", "WF_ERR_STAGE_ORDER", "WF_ERR_CAPACITY",
+    "WF_ERR_PAGE_OOB", "WF_ERR_TIMEOUT", "WF_ERR_CUDA", "WF_ERR_NO_DEVICE", "WF_MAX_CHUNKS",
+    "WavefrontDesc", "WfError", "attn_forward", "check_status", "kv_append", "strerror",
+)
+__all__ = list(_ABI_NAMES)
+
+
+def __getattr__(name):
+    if name in _ABI_NAMES:
+        from . import _abi
+        return getattr(_abi, name)
+    raise AttributeError(name)

@@ -1,0 +1,156 @@
+"""ctypes binding of ``libwf_b200.so`` (the C ABI in ``include/wf.h``).
+
+Argument marshalling only: every step of append and attention runs in the library's kernels.
+There is no CPU fallback; if the library is missing, importing the binding raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libwf_b200.so")
+
+WF_OK = 0
+WF_ERR_INVALID_ARG = 1
+WF_ERR_SHAPE = 2
+WF_ERR_STAGE_ORDER = 3
+WF_ERR_CAPACITY = 4
+WF_ERR_PAGE_OOB = 5
+WF_ERR_TIMEOUT = 6
+WF_ERR_CUDA = 7
+WF_ERR_NO_DEVICE = 8
+WF_MAX_CHUNKS = 64
+
+# Every symbol include/wf.h declares (checked by the CPU tests).
+EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror", "wf_version")
+
+
+class WfError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code)}")
+
+
+class KvPool(ctypes.Structure):
+    _fields_ = [("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p),
+                ("num_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+class Wavefront(ctypes.Structure):
+    _fields_ = [("num_chunks", ctypes.c_int32), ("num_ctx_chunks", ctypes.c_int32),
+                ("chunk_offsets", ctypes.POINTER(ctypes.c_int32)),
+                ("chunk_stage", ctypes.POINTER(ctypes.c_int32)),
+                ("max_pages_per_seq", ctypes.c_int32)]
+
+
+def _load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m block_causal_streaming_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.wf_kv_append.argtypes = [ctypes.POINTER(KvPool), i32, i32, vp, vp,
+                                 ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(Wavefront), vp]
+    lib.wf_kv_append.restype = i32
+    lib.wf_attn_forward.argtypes = [vp, ctypes.POINTER(KvPool), ctypes.POINTER(ctypes.c_int32),
+                                    ctypes.POINTER(Wavefront), f32, vp,
+                                    ctypes.POINTER(ctypes.c_float), vp]
+    lib.wf_attn_forward.restype = i32
+    lib.wf_check_status.argtypes = [vp]
+    lib.wf_check_status.restype = i32
+    lib.wf_strerror.argtypes = [i32]
+    lib.wf_strerror.restype = ctypes.c_char_p
+    lib.wf_version.argtypes = []
+    lib.wf_version.restype = i32
+    return lib
+
+
+lib = _load()
+
+
+def strerror(code: int) -> str:
+    return lib.wf_strerror(int(code)).decode()
+
+
+class WavefrontDesc:
+    """Host copy of a wavefront descriptor; keeps the arrays alive while C reads them."""
+
+    def __init__(self, chunk_offsets: Sequence[int], chunk_stage: Sequence[int],
+                 num_ctx_chunks: int, max_pages_per_seq: int):
+        n = len(chunk_offsets) - 1
+        self._off = (ctypes.c_int32 * (n + 1))(*[int(x) for x in chunk_offsets])
+        self._stage = (ctypes.c_int32 * max(n, 1))(*[int(x) for x in chunk_stage])
+        self.c = Wavefront(n, int(num_ctx_chunks),
+                           ctypes.cast(self._off, ctypes.POINTER(ctypes.c_int32)),
+                           ctypes.cast(self._stage, ctypes.POINTER(ctypes.c_int32)),
+                           int(max_pages_per_seq))
+        self.chunk_offsets = [int(x) for x in chunk_offsets]
+        self.num_ctx_chunks = int(num_ctx_chunks)
+
+
+def _pool_struct(k_pool, v_pool) -> KvPool:
+    num_pages, page_size, H, D = (int(x) for x in k_pool.shape)
+    return KvPool(k_pool.data_ptr(), v_pool.data_ptr(), num_pages, page_size, H, D)
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _check_tensor(t, name: str, dtype_name: str):
+    import torch
+    want = {"bf16": torch.bfloat16, "i32": torch.int32, "f32": torch.float32}[dtype_name]
+    if t.dtype != want:
+        raise TypeError(f"{name}: expected {want}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+
+
+def kv_append(k_pool, v_pool, layer: int, chunk: int, k, v, page_table, wf: WavefrontDesc,
+              stream=None) -> None:
+    """wf_kv_append: write chunk ``chunk``'s K/V ([L, H, D] bf16) into the pools' pages using row
+    ``layer`` of ``page_table`` ([num_layers, max_pages_per_seq] int32, on the device)."""
+    for t, n, d in ((k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"), (k, "k", "bf16"),
+                    (v, "v", "bf16"), (page_table, "page_table", "i32")):
+        _check_tensor(t, n, d)
+    pool = _pool_struct(k_pool, v_pool)
+    rc = lib.wf_kv_append(ctypes.byref(pool), int(layer), int(chunk), k.data_ptr(), v.data_ptr(),
+                          ctypes.cast(ctypes.c_void_p(page_table.data_ptr()),
+                                      ctypes.POINTER(ctypes.c_int32)),
+                          ctypes.byref(wf.c), _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_kv_append")
+
+
+def attn_forward(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: float, out,
+                 lse=None, stream=None) -> None:
+    """wf_attn_forward: block-causal chunk attention of q ([T_q, H, D] bf16) over the paged K/V
+    of one layer (``page_table_row``: [max_pages_per_seq] int32 on the device) into ``out``."""
+    for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
+                    (page_table_row, "page_table_row", "i32"), (out, "out", "bf16")):
+        _check_tensor(t, n, d)
+    if lse is not None:
+        _check_tensor(lse, "lse", "f32")
+    pool = _pool_struct(k_pool, v_pool)
+    rc = lib.wf_attn_forward(
+        q.data_ptr(), ctypes.byref(pool),
+        ctypes.cast(ctypes.c_void_p(page_table_row.data_ptr()), ctypes.POINTER(ctypes.c_int32)),
+        ctypes.byref(wf.c), float(scale), out.data_ptr(),
+        ctypes.cast(ctypes.c_void_p(lse.data_ptr()), ctypes.POINTER(ctypes.c_float))
+        if lse is not None else None,
+        _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_attn_forward")
+
+
+def check_status(stream=None) -> int:
+    """wf_check_status: synchronise the stream and return (and clear) the first device error."""
+    return int(lib.wf_check_status(_stream_handle(stream)))

@@ -1,0 +1,56 @@
+"""Build the in-tree CUDA library ``libwf_b200.so`` for sm_100a (nvcc cross-compiles; no GPU needed).
+
+    python -m block_causal_streaming_b200.build [-v]
+
+The library is one translation unit (``csrc/wf_api.cu``, which includes the kernels) linked
+against the static CUDA runtime, so it only needs the driver at run time.
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+LIB = os.path.join(HERE, "libwf_b200.so")
+SOURCES = [os.path.join(CSRC, "wf_api.cu")]
+DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "attn_kernel.cuh",
+                                                      "append_kernel.cuh")] + \
+    [os.path.join(ROOT, "include", "wf.h")]
+
+NVCC_FLAGS = [
+    "-O3", "-std=c++17", "-lineinfo",
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-shared", "-Xcompiler", "-fPIC", "-cudart", "static",
+    "-I" + os.path.join(ROOT, "include"),
+]
+
+
+def nvcc() -> str:
+    cand = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
+    return cand if os.path.exists(cand) else "nvcc"
+
+
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
+        return True
+    t = os.path.getmtime(lib)
+    return any(os.path.getmtime(f) > t for f in DEPENDS if os.path.exists(f))
+
+
+def build(verbose: bool = False, force: bool = False, out: str = LIB) -> str:
+    if not force and not needs_build(out):
+        return out
+    cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + SOURCES + ["-o", out]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if verbose or res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+    if res.returncode != 0:
+        raise RuntimeError(f"nvcc failed ({res.returncode}): {' '.join(cmd)}")
+    return out
+
+
+if __name__ == "__main__":
+    print(build(verbose="-v" in sys.argv, force=True))

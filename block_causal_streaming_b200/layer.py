@@ -1,0 +1,69 @@
+"""Device-side state of one wavefront layer: paged K/V pools, page table and descriptor.
+
+PyTorch provides the device memory and the stream; every step of the hot path runs through the
+C ABI (:mod:`._abi`).  A pool may be shared by several layers (each with its own page-table row),
+which is how the 30-layer round reuses one 4096-page pool.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import torch
+
+from . import _abi
+
+
+class PagedPool:
+    """K and V pools, bf16 [num_pages, page_size, H, D] each, on one device."""
+
+    def __init__(self, num_pages: int, page_size: int, heads: int, head_dim: int,
+                 device="cuda", fill: Optional[float] = None):
+        shape = (num_pages, page_size, heads, head_dim)
+        self.k = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        self.v = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        if fill is not None:
+            self.k.fill_(fill)
+            self.v.fill_(fill)
+        self.num_pages, self.page_size, self.heads, self.head_dim = shape
+
+
+class WavefrontLayer:
+    """One layer of a wavefront: its descriptor and its page-table rows.
+
+    ``page_tables`` is int32 [num_layers, max_pages_per_seq] on the device (row ``layer`` is this
+    layer's); ``chunk_offsets`` / ``chunk_stage`` / ``num_ctx_chunks`` describe the chunks in
+    logical order (context first, then active chunks cleanest to noisiest).
+    """
+
+    def __init__(self, pool: PagedPool, page_tables: torch.Tensor, layer: int,
+                 chunk_offsets: Sequence[int], chunk_stage: Sequence[int], num_ctx_chunks: int):
+        self.pool = pool
+        self.page_tables = page_tables
+        self.layer = int(layer)
+        self.desc = _abi.WavefrontDesc(chunk_offsets, chunk_stage, num_ctx_chunks,
+                                       page_tables.shape[1])
+        self.chunk_offsets = list(chunk_offsets)
+        self.num_ctx_chunks = int(num_ctx_chunks)
+
+    @property
+    def t_q(self) -> int:
+        return self.chunk_offsets[-1] - self.chunk_offsets[self.num_ctx_chunks]
+
+    def append(self, chunk: int, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
+        _abi.kv_append(self.pool.k, self.pool.v, self.layer, chunk, k, v, self.page_tables,
+                       self.desc, stream)
+
+    def append_range(self, k_all: torch.Tensor, v_all: torch.Tensor, chunks: Sequence[int],
+                     stream=None) -> None:
+        """Append the given chunks, slicing their rows out of logical-order K/V tensors."""
+        for c in chunks:
+            a, b = self.chunk_offsets[c], self.chunk_offsets[c + 1]
+            self.append(c, k_all[a:b], v_all[a:b], stream)
+
+    def forward(self, q: torch.Tensor, out: torch.Tensor, scale: Optional[float] = None,
+                lse: Optional[torch.Tensor] = None, stream=None) -> None:
+        if scale is None:
+            scale = 1.0 / math.sqrt(self.pool.head_dim)
+        _abi.attn_forward(q, self.pool.k, self.pool.v, self.page_tables[self.layer], self.desc,
+                          scale, out, lse, stream)

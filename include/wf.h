@@ -1,0 +1,150 @@
+/*
+ * wf.h -- C ABI of the B200 (sm_100a) block-causal chunk-attention library for Wave Forcing.
+ *
+ * Wave Forcing runs a DiT over a mixed-noise wavefront of video chunks.  Inside every Transformer
+ * layer, the queries of each active chunk attend fully within their own chunk and, across chunks,
+ * only to earlier, cleaner chunks -- the anchor, the clean history and earlier in-flight chunks --
+ * and never to a later, noisier one (KipQuest summary of arXiv 2611.00859, "The deep dive",
+ * paragraph on chunk-wise causal attention; project page, "01 The design gap", panel C).
+ * The K/V of every chunk is published once per layer into fixed slots of the consumer's attention
+ * buffer, and attention reads its visible prefix in place with no concatenation (project page,
+ * "03 End-to-end KV transport", item 03 "Layout"; the README's "paged" exchange mode).  This
+ * library holds those slots in fixed-size pages addressed through a page table.
+ *
+ * Logical order.  The K/V sequence of one layer is the chunks in order oldest (cleanest) first:
+ * KV-only context chunks (anchor, clean history; stage 0), then the active chunks from the
+ * cleanest to the noisiest.  Chunk c owns logical tokens [chunk_offsets[c], chunk_offsets[c+1]).
+ * With this order the keys a query of chunk c may see are exactly the prefix
+ * [0, chunk_offsets[c+1]).
+ *
+ * Paged layout.  K and V pools are bf16 arrays [num_pages][page_size][num_heads][head_dim]
+ * (row-major, contiguous).  Logical token t of a layer lives in physical page
+ * page_table_row[t / page_size] at row t % page_size.  Chunks are packed token-contiguously, so
+ * one page may hold the tail of one chunk and the head of the next.
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are CUDA device memory on the current device; "host" pointers are
+ *     read during the call only.  The caller owns every buffer; the library keeps no pointer after
+ *     a call returns.
+ *   - Calls are asynchronous on the given stream (0 = legacy default stream) and never
+ *     synchronise, except wf_check_status.
+ *   - Every call returns WF_OK (0) or an error code; nothing else crosses the ABI.  Argument
+ *     errors are detected on the host before anything is launched.  Errors found by a kernel
+ *     (a page index outside the pool, a bounded wait that ran out) are recorded in a per-device
+ *     status word read by wf_check_status.
+ *   - bf16 only, batch 1, one layer per call.
+ */
+#ifndef WF_H_
+#define WF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* wf_stream_t; /* a cudaStream_t */
+
+enum {
+  WF_OK = 0,
+  WF_ERR_INVALID_ARG = 1,  /* null or misaligned pointer, layer/chunk index out of range, scale <= 0 */
+  WF_ERR_SHAPE = 2,        /* head_dim not 64/128, page_size not a positive multiple of 16,
+                              offsets not starting at 0 or decreasing, too many chunks, no query chunk */
+  WF_ERR_STAGE_ORDER = 3,  /* chunk_stage decreases along the logical (oldest-first) order */
+  WF_ERR_CAPACITY = 4,     /* the layer needs more pages than max_pages_per_seq */
+  WF_ERR_PAGE_OOB = 5,     /* device: a page-table entry outside [0, num_pages); that page was not
+                              written (append) or was read as page 0 (attention) */
+  WF_ERR_TIMEOUT = 6,      /* device: a bounded wait inside a kernel ran out; the kernel stopped */
+  WF_ERR_CUDA = 7,         /* a CUDA runtime or driver call failed */
+  WF_ERR_NO_DEVICE = 8     /* no sm_100 device is current */
+};
+
+/* Maximum number of chunks (context + active) in one wavefront descriptor. */
+#define WF_MAX_CHUNKS 64
+
+/* One layer-independent K/V pool.  k_pool, v_pool: device bf16 [num_pages][page_size][H][D],
+ * 16-byte aligned, caller-owned. */
+typedef struct {
+  void* k_pool;
+  void* v_pool;
+  int32_t num_pages;
+  int32_t page_size;   /* tokens per page: a positive multiple of 16 */
+  int32_t num_heads;
+  int32_t head_dim;    /* 64 or 128 */
+} wf_kv_pool_t;
+
+/* The wavefront: which chunks exist, where their tokens sit, and their diffusion stage. */
+typedef struct {
+  int32_t num_chunks;          /* context + active, 1..WF_MAX_CHUNKS */
+  int32_t num_ctx_chunks;      /* leading KV-only chunks; queries exist for chunks >= this */
+  const int32_t* chunk_offsets;/* host [num_chunks+1]: token offsets in the logical sequence,
+                                  [0] = 0, non-decreasing (an empty chunk is allowed) */
+  const int32_t* chunk_stage;  /* host [num_chunks]: diffusion timestep, 0 = clean; must be
+                                  non-decreasing in logical order (earlier = cleaner).  Validated
+                                  only; the mask follows the logical order. */
+  int32_t max_pages_per_seq;   /* row length of the page table */
+} wf_wavefront_t;
+
+/*
+ * wf_kv_append -- publish one chunk's K/V of one layer into its pages.
+ * Defining passage: project page, "03 End-to-end KV transport", item 03 "Layout" (each producer
+ * writes straight into its fixed slot of the consumer's attention buffer); KipQuest "The deep
+ * dive" (each replica publishes its keys and values right after projection, at every layer).
+ *
+ *   pool        K/V pools (device).
+ *   layer       row of page_table to use, >= 0.
+ *   chunk       chunk index in [0, wf->num_chunks).
+ *   k, v        device bf16 [L][H][D], contiguous, 16-byte aligned, L = chunk length.
+ *   page_table  device int32 [num_layers][max_pages_per_seq]; row `layer` maps logical pages of
+ *               that layer to physical pages.
+ *   wf          the wavefront (host).
+ * Copies token i of the chunk to logical token chunk_offsets[chunk] + i, bit for bit.  Rows of a
+ * page outside the chunk are not touched.  An entry outside [0, num_pages) is skipped and
+ * recorded as WF_ERR_PAGE_OOB.  An empty chunk is a no-op.
+ */
+int wf_kv_append(const wf_kv_pool_t* pool, int layer, int chunk, const void* k, const void* v,
+                 const int32_t* page_table, const wf_wavefront_t* wf, wf_stream_t stream);
+
+/*
+ * wf_attn_forward -- one block-causal chunk attention over the whole wavefront, one launch.
+ * Defining passages: KipQuest "The deep dive" (within a chunk full; across chunks the anchor,
+ * the clean history and every earlier, cleaner chunk, never a later, noisier one); project page
+ * "01 The design gap" panel C; "03 End-to-end KV transport" item 03 (attention reads the prefix in
+ * place).
+ *
+ *   q               device bf16 [T_q][H][D]: the query rows of chunks num_ctx_chunks..num_chunks-1
+ *                   in order, T_q = chunk_offsets[num_chunks] - chunk_offsets[num_ctx_chunks].
+ *   kv_pages        the K/V pools (device); every token in [0, chunk_offsets[num_chunks]) must
+ *                   have been appended.  Rows past the last token may hold anything, NaN included.
+ *   page_table_row  device int32 [max_pages_per_seq]: ONE layer's row.
+ *   wf              the wavefront (host).
+ *   scale           softmax scale (> 0), typically 1/sqrt(head_dim).
+ *   out             device bf16 [T_q][H][D]: out[t,h,:] = sum_j softmax_j(scale q.k_j) v_j over
+ *                   the keys j < chunk_offsets[c+1] of the query's chunk c.  fp32 accumulation,
+ *                   P rounded to bf16 before P.V, output rounded to nearest even.
+ *   lse_or_null     device fp32 [H][T_q] (optional): natural-log sum of exp of the scaled logits.
+ * T_q = 0 is a no-op.
+ */
+int wf_attn_forward(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* page_table_row,
+                    const wf_wavefront_t* wf, float scale, void* out, float* lse_or_null,
+                    wf_stream_t stream);
+
+/*
+ * wf_check_status -- synchronise `stream`, then return and clear the first error any kernel of
+ * this library recorded on the current device since the last call (WF_OK if none).  A pending
+ * CUDA error on the stream is returned as WF_ERR_CUDA.
+ */
+int wf_check_status(wf_stream_t stream);
+
+/* wf_strerror -- a static, human-readable name for an error code. */
+const char* wf_strerror(int code);
+
+/* wf_version -- library version, major * 10000 + minor * 100 + patch. */
+int wf_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WF_H_ */

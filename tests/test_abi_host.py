@@ -1,0 +1,119 @@
+"""The C-ABI library on the host: it loads, exports exactly what include/wf.h declares, and its
+argument validation answers before anything touches a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from block_causal_streaming_b200 import build as wf_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wf.h")
+
+
+@pytest.fixture(scope="module")
+def abi():
+    wf_build.build()
+    from block_causal_streaming_b200 import _abi
+    return _abi
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(wf_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declarations_match_binding(abi):
+    assert declared_functions() == sorted(abi.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(abi):
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} is declared but not exported"
+
+
+def test_header_error_codes_match_binding(abi):
+    text = open(HEADER).read()
+    codes = dict((m.group(1), int(m.group(2)))
+                 for m in re.finditer(r"(WF_(?:OK|ERR_\w+))\s*=\s*(\d+)", text))
+    for name, value in codes.items():
+        assert getattr(abi, name) == value, name
+    assert abi.WF_MAX_CHUNKS == int(re.search(r"#define WF_MAX_CHUNKS (\d+)", text).group(1))
+
+
+def test_strerror_and_version(abi):
+    for code in range(0, 9):
+        assert abi.strerror(code).startswith("WF_")
+    assert "unknown" in abi.strerror(99)
+    assert abi.lib.wf_version() >= 100
+
+
+FAKE = 0x10000  # an aligned, never-dereferenced address: validation must answer first
+
+
+def _pool(abi, **kw):
+    args = dict(k_pool=FAKE, v_pool=FAKE, num_pages=8, page_size=64, num_heads=2, head_dim=128)
+    args.update(kw)
+    return abi.KvPool(**args)
+
+
+def _attn(abi, pool, desc, scale=0.1, q=FAKE, out=FAKE, pt=FAKE):
+    return abi.lib.wf_attn_forward(q, ctypes.byref(pool),
+                                   ctypes.cast(ctypes.c_void_p(pt), ctypes.POINTER(ctypes.c_int32)),
+                                   ctypes.byref(desc.c), scale, out, None, None)
+
+
+def _append(abi, pool, desc, layer=0, chunk=0, k=FAKE, v=FAKE, pt=FAKE):
+    return abi.lib.wf_kv_append(ctypes.byref(pool), layer, chunk, k, v,
+                                ctypes.cast(ctypes.c_void_p(pt), ctypes.POINTER(ctypes.c_int32)),
+                                ctypes.byref(desc.c), None)
+
+
+def test_validation_errors_without_a_gpu(abi):
+    ok_desc = abi.WavefrontDesc([0, 64, 128, 200], [0, 200, 1000], 1, 8)
+    # pool checks
+    assert _attn(abi, _pool(abi, k_pool=0), ok_desc) == abi.WF_ERR_INVALID_ARG
+    assert _attn(abi, _pool(abi, v_pool=FAKE + 8), ok_desc) == abi.WF_ERR_INVALID_ARG
+    assert _attn(abi, _pool(abi, head_dim=96), ok_desc) == abi.WF_ERR_SHAPE
+    assert _attn(abi, _pool(abi, page_size=24), ok_desc) == abi.WF_ERR_SHAPE
+    assert _attn(abi, _pool(abi, page_size=0), ok_desc) == abi.WF_ERR_SHAPE
+    assert _attn(abi, _pool(abi, num_heads=0), ok_desc) == abi.WF_ERR_SHAPE
+    # descriptor checks
+    assert _attn(abi, _pool(abi), abi.WavefrontDesc([1, 64, 128], [0, 0], 0, 8)) == \
+        abi.WF_ERR_SHAPE
+    assert _attn(abi, _pool(abi), abi.WavefrontDesc([0, 64, 60], [0, 0], 0, 8)) == \
+        abi.WF_ERR_SHAPE
+    assert _attn(abi, _pool(abi), abi.WavefrontDesc([0, 64, 128], [500, 200], 0, 8)) == \
+        abi.WF_ERR_STAGE_ORDER
+    assert _attn(abi, _pool(abi), abi.WavefrontDesc([0, 64, 600], [0, 0], 0, 8)) == \
+        abi.WF_ERR_CAPACITY
+    assert _attn(abi, _pool(abi), abi.WavefrontDesc([0, 64, 128], [0, 0], 2, 8)) == \
+        abi.WF_ERR_SHAPE                                          # no query chunk
+    too_many = list(range(0, 66))
+    assert _attn(abi, _pool(abi), abi.WavefrontDesc(too_many, [0] * 65, 0, 8)) == \
+        abi.WF_ERR_SHAPE
+    # call arguments
+    assert _attn(abi, _pool(abi), ok_desc, scale=0.0) == abi.WF_ERR_INVALID_ARG
+    assert _attn(abi, _pool(abi), ok_desc, scale=float("nan")) == abi.WF_ERR_INVALID_ARG
+    assert _attn(abi, _pool(abi), ok_desc, q=0) == abi.WF_ERR_INVALID_ARG
+    assert _attn(abi, _pool(abi), ok_desc, out=FAKE + 2) == abi.WF_ERR_INVALID_ARG
+    assert _append(abi, _pool(abi), ok_desc, chunk=3) == abi.WF_ERR_INVALID_ARG
+    assert _append(abi, _pool(abi), ok_desc, layer=-1) == abi.WF_ERR_INVALID_ARG
+    assert _append(abi, _pool(abi), ok_desc, k=FAKE + 4) == abi.WF_ERR_INVALID_ARG
+
+
+def test_empty_work_is_a_no_op(abi):
+    """T_q = 0 and empty chunks return WF_OK before any device work."""
+    desc = abi.WavefrontDesc([0, 64, 64], [0, 0], 1, 8)        # the only query chunk is empty
+    assert _attn(abi, _pool(abi), desc) == abi.WF_OK
+    assert _append(abi, _pool(abi), desc, chunk=1) == abi.WF_OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device answer")
+def test_valid_call_without_device_reports_no_device(abi):
+    desc = abi.WavefrontDesc([0, 64, 128, 200], [0, 200, 1000], 1, 8)
+    assert _attn(abi, _pool(abi), desc) == abi.WF_ERR_NO_DEVICE
+    assert _append(abi, _pool(abi), desc) == abi.WF_ERR_NO_DEVICE

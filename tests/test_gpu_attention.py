@@ -1,0 +1,184 @@
+"""wf_attn_forward on the GPU against the oracle.
+
+Parity bar (stated by the build's target): max-abs <= 1e-2 and mean-abs <= 1e-3 on bf16 outputs
+with fp32 accumulation.  Small cases are compared element by element on every output; the five
+benchmark workloads are compared on sampled rows (chunk edges, tile edges, the tail) plus
+properties that hold at any size.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_causal_streaming_b200 import WF_ERR_PAGE_OOB, WF_OK, check_status
+from block_causal_streaming_b200.workloads import (CONFIGS, LayerInputs, make_inputs, make_layers,
+                                                   small_case)
+from gpu_util import assert_parity, place, run, sample_rows, scale_of
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    small_case("d128_ps64_ctx2_act3", 2, 128, (300, 200), (257, 300, 129), 64, seed=11),
+    small_case("d64_ps16_noctx", 3, 64, (), (48, 48, 48, 100), 16, seed=12),
+    small_case("d128_ps48_short_chunks", 1, 128, (37,), (5, 1, 130, 70), 48, seed=13),
+    small_case("d128_ps256_single_chunk", 2, 128, (), (700,), 256, seed=14),
+    small_case("d128_ps128_tq_below_tile", 2, 128, (500,), (20,), 128, seed=15),
+    small_case("d64_ps32_many_chunks", 2, 64, (64, 64, 64), (33, 95, 128, 256, 1), 32, seed=16),
+    small_case("d128_kmean", 2, 128, (400, 400), (300, 300), 64, seed=17, k_mean_offset=True),
+    small_case("d128_empty_active_chunk", 2, 128, (90,), (100, 0, 50), 16, seed=18),
+    small_case("d64_ps128_pool_larger", 4, 64, (130,), (250, 260), 128, seed=19, pool_pages=20),
+]
+
+
+def full_oracle(wl, inp, with_lse=True):
+    return oracle.attention(inp.q, inp.k, inp.v, wl.chunk_offsets, wl.num_ctx_chunks,
+                            scale_of(wl), with_lse=with_lse)
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_small_parity_every_element(wl):
+    inp = make_inputs(wl)
+    layer, q, _, _ = place(wl, inp, fill=float("nan"), extra_pages=2)
+    out, lse = run(layer, q, with_lse=True)
+    assert check_status() == WF_OK
+    ref, ref_lse = full_oracle(wl, inp)
+    assert_parity(out.float().cpu().numpy(), ref, wl.name)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=2e-3)
+
+
+def test_config1_tiny_every_element():
+    wl = CONFIGS[1]
+    inp = make_inputs(wl)
+    layer, q, _, _ = place(wl, inp)
+    out = run(layer, q)
+    assert check_status() == WF_OK
+    assert_parity(out.float().cpu().numpy(), full_oracle(wl, inp, with_lse=False), wl.name)
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 5])
+def test_full_size_config_sampled_parity(cfg):
+    wl = CONFIGS[cfg]
+    inp = make_inputs(wl)
+    layer, q, _, _ = place(wl, inp, fill=float("nan"))
+    out, lse = run(layer, q, with_lse=True)
+    out2 = run(layer, q)
+    assert check_status() == WF_OK
+    assert torch.equal(out, out2), "two identical runs differ"
+    assert torch.isfinite(out.float()).all()
+    rows, heads = sample_rows(wl, per_chunk=4, seed=cfg)
+    ref, ref_lse = oracle.attention_rows(inp.q, inp.k, inp.v, wl.chunk_offsets,
+                                         wl.num_ctx_chunks, scale_of(wl), rows, heads,
+                                         with_lse=True)
+    got = out[rows, heads].float().cpu().numpy()
+    assert_parity(got, ref, wl.name)
+    np.testing.assert_allclose(lse[heads, rows].cpu().numpy(), ref_lse, rtol=0, atol=2e-3)
+
+
+def test_config4_thirty_layer_round_sampled_parity():
+    """30 layers share one 4096-page pool; each layer appends its chunks, then attends."""
+    wl = CONFIGS[4]
+    layers = make_layers(wl)
+    from block_causal_streaming_b200.layer import PagedPool, WavefrontLayer
+    pool = PagedPool(wl.num_pages, wl.page_size, wl.heads, wl.head_dim, "cuda")
+    pts = torch.stack([l.page_table for l in layers]).cuda()
+    outs = []
+    for i, inp in enumerate(layers):
+        layer = WavefrontLayer(pool, pts, i, wl.chunk_offsets, wl.chunk_stage, wl.num_ctx_chunks)
+        layer.append_range(inp.k.cuda(), inp.v.cuda(), range(wl.num_chunks))
+        outs.append(run(layer, inp.q.cuda()).cpu())
+    assert check_status() == WF_OK
+    for i, inp in enumerate(layers):
+        rows, heads = sample_rows(wl, per_chunk=1, seed=100 + i)
+        ref = oracle.attention_rows(inp.q, inp.k, inp.v, wl.chunk_offsets, wl.num_ctx_chunks,
+                                    scale_of(wl), rows, heads)
+        assert_parity(outs[i][rows, heads].float().numpy(), ref, f"layer {i}")
+
+
+# ------------------------------------------------------------------------------- invariants
+MED = small_case("invariants", 2, 128, (300,), (200, 300, 250), 64, seed=21)
+
+
+def test_later_chunks_are_invisible_bitwise():
+    wl = MED
+    inp = make_inputs(wl)
+    layer, q, k, v = place(wl, inp)
+    base = run(layer, q)
+    off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
+    for i in range(nctx, wl.num_chunks - 1):
+        k2, v2 = k.clone(), v.clone()
+        k2[off[i + 1]:] = torch.randn_like(k2[off[i + 1]:].float()).to(torch.bfloat16) * 5
+        v2[off[i + 1]:] = torch.randn_like(v2[off[i + 1]:].float()).to(torch.bfloat16) * 5
+        layer.append_range(k2, v2, range(i + 1, wl.num_chunks))
+        got = run(layer, q)
+        rows = off[i + 1] - off[nctx]
+        assert torch.equal(got[:rows], base[:rows]), f"chunk <= {i} changed"
+        assert not torch.equal(got[rows:], base[rows:])
+        layer.append_range(k, v, range(i + 1, wl.num_chunks))   # restore
+    assert check_status() == WF_OK
+
+
+def test_values_of_later_chunks_never_leak():
+    wl = MED
+    inp = make_inputs(wl)
+    off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
+    for j in range(nctx + 1, wl.num_chunks):
+        v = torch.zeros_like(inp.v)
+        v[off[j]:off[j + 1]] = inp.v[off[j]:off[j + 1]]
+        layer, q, _, _ = place(wl, LayerInputs(inp.q, inp.k, v, inp.page_table))
+        out = run(layer, q)
+        before = off[j] - off[nctx]
+        assert torch.all(out[:before] == 0), f"chunk {j}'s values leaked into earlier chunks"
+        assert torch.any(out[before:off[j + 1] - off[nctx]] != 0)
+    assert check_status() == WF_OK
+
+
+def test_zero_queries_give_prefix_mean():
+    wl = MED
+    inp = make_inputs(wl)
+    inp = LayerInputs(torch.zeros_like(inp.q), inp.k, inp.v, inp.page_table)
+    layer, q, _, _ = place(wl, inp)
+    out, lse = run(layer, q, with_lse=True)
+    off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
+    csum = torch.cat([torch.zeros(1, wl.heads, wl.head_dim, dtype=torch.float64),
+                      inp.v.double().cumsum(0)])
+    for c in range(nctx, wl.num_chunks):
+        n = off[c + 1]
+        rows = slice(off[c] - off[nctx], off[c + 1] - off[nctx])
+        mean = (csum[n] / n).float()
+        err = (out[rows].float().cpu() - mean).abs().max().item()
+        assert err <= 1e-2, f"chunk {c}: prefix-mean error {err}"
+        assert (lse[:, rows].cpu() - math.log(n)).abs().max().item() <= 1e-3
+
+
+def test_unit_values_give_unit_outputs():
+    wl = small_case("unit_v", 3, 128, (1000,), (600, 700), 64, seed=22, value_scale=2.0)
+    inp = make_inputs(wl)
+    inp = LayerInputs(inp.q, inp.k, torch.ones_like(inp.v), inp.page_table)
+    layer, q, _, _ = place(wl, inp, fill=float("nan"))
+    out = run(layer, q)
+    assert (out.float() - 1).abs().max().item() <= 1e-3
+
+
+def test_page_permutation_is_invisible_bitwise():
+    wl = MED
+    inp = make_inputs(wl)
+    ident = LayerInputs(inp.q, inp.k, inp.v, torch.arange(wl.pages_needed, dtype=torch.int32))
+    perm = LayerInputs(inp.q, inp.k, inp.v,
+                       torch.randperm(wl.pages_needed + 9,
+                                      generator=torch.Generator().manual_seed(3))[
+                           :wl.pages_needed].to(torch.int32))
+    layer_a, q, _, _ = place(wl, ident)
+    layer_b, _, _, _ = place(wl, perm, extra_pages=9, fill=float("nan"))
+    assert torch.equal(run(layer_a, q), run(layer_b, q))
+
+
+def test_out_of_range_page_in_attention_is_reported():
+    wl = small_case("oob_attn", 1, 128, (64,), (64,), 64, seed=23)
+    inp = make_inputs(wl)
+    layer, q, _, _ = place(wl, inp)
+    layer.page_tables[0, 1] = 99                     # outside the 2-page pool
+    run(layer, q)
+    assert check_status() == WF_ERR_PAGE_OOB
+    assert check_status() == WF_OK
