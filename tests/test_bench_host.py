@@ -1,0 +1,82 @@
+"""Host logic of bench.py: FLOP accounting, replica aggregation and max-over-ranks timing, with
+world-size-2 gloo process groups on the CPU."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from block_causal_streaming_b200.workloads import CONFIGS, small_case
+
+
+def _visible_pairs(wl):
+    """Count (query, key) pairs allowed by the mask rule, by brute force over chunk indices."""
+    off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
+    ids = np.concatenate([np.full(off[c + 1] - off[c], c) for c in range(wl.num_chunks)])
+    q_ids = ids[off[nctx]:]
+    return int((ids[None, :] <= q_ids[:, None]).sum())
+
+
+@pytest.mark.parametrize("wl", [CONFIGS[1],
+                                small_case("acct", 3, 128, (50, 7), (33, 0, 90), 16, seed=1),
+                                small_case("acct2", 2, 64, (), (300,), 64, seed=2)],
+                         ids=lambda w: w.name)
+def test_flop_accounting_counts_only_visible_pairs(wl):
+    assert bench.attention_flops(wl) == 4 * wl.head_dim * wl.heads * _visible_pairs(wl)
+
+
+def test_flop_accounting_of_benchmark_workloads():
+    # 4*D*H*sum(len_c * end_c): 5 chunks of 4680 after 2 context chunks, H=12, D=128
+    assert bench.attention_flops(CONFIGS[2]) == 4 * 128 * 12 * sum(
+        4680 * 4680 * (c + 1) for c in range(2, 7))
+
+
+def test_row_flops_matches_total():
+    wl = CONFIGS[1]
+    assert bench.rows_flops(wl, range(wl.t_q), wl.heads) == bench.attention_flops(wl)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    bench.init_dist(world, "gloo")
+    try:
+        bench.barrier(world)
+        t = bench.max_over_ranks(1.0 + rank, world)       # rank 1 is the slower one
+        results[rank] = (t, bench.aggregate(10.0, world, t))
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replicas_take_the_slowest_rank_gloo():
+    world = 2
+    with mp.Manager() as m:
+        results = m.dict()
+        mp.start_processes(_rank_main, args=(world, _free_port(), results), nprocs=world,
+                           start_method="spawn", join=True)
+        got = dict(results)
+    assert got[0] == got[1] == (2.0, 10.0)     # 2 ranks x 10 units / 2.0 s
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
+    class A:
+        config, steps, warmup, cpu_seconds = 2, 1, 3, 1.0
+    assert bench.reference_arm(A, world=2, rank=1) is None
+
+
+def test_arguments_are_checked():
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2"])
