@@ -10,7 +10,8 @@ import os
 from typing import Optional, Sequence
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libwf_b200.so")
+# WF_B200_LIB points the binding at another build of the same library (e.g. a tuning variant).
+LIB_PATH = os.environ.get("WF_B200_LIB") or os.path.join(HERE, "libwf_b200.so")
 
 WF_OK = 0
 WF_ERR_INVALID_ARG = 1

@@ -8,6 +8,7 @@ against the static CUDA runtime, so it only needs the driver at run time.
 from __future__ import annotations
 
 import os
+import re
 import subprocess
 import sys
 
@@ -40,15 +41,45 @@ def needs_build(lib: str = LIB) -> bool:
     return any(os.path.getmtime(f) > t for f in DEPENDS if os.path.exists(f))
 
 
+# The attention kernel splits its register file with setmaxnreg assuming it is launched with
+# 168 registers per thread (384 threads); a different count would make the split wait forever.
+ATTN_LAUNCH_REGS = 168
+
+
+def check_register_counts(ptxas_log: str) -> None:
+    """Fail the build unless every attention kernel was compiled for ATTN_LAUNCH_REGS."""
+    entry = None
+    found = 0
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            entry = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and entry and "wf_attn_fwd_kernel" in entry:
+            found += 1
+            if int(m.group(1)) != ATTN_LAUNCH_REGS:
+                raise RuntimeError(f"{entry}: {m.group(1)} registers, expected {ATTN_LAUNCH_REGS}"
+                                   " (the setmaxnreg split in attn_kernel.cuh depends on it)")
+            entry = None
+    if found == 0:
+        raise RuntimeError("ptxas reported no attention kernel")
+
+
 def build(verbose: bool = False, force: bool = False, out: str = LIB) -> str:
     if not force and not needs_build(out):
         return out
-    cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + SOURCES + ["-o", out]
+    cmd = [nvcc()] + NVCC_FLAGS + ["-Xptxas", "-v"] + SOURCES + ["-o", out]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if verbose or res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed ({res.returncode}): {' '.join(cmd)}")
+    try:
+        check_register_counts(res.stdout + res.stderr)
+    except RuntimeError:
+        os.remove(out)
+        raise
     return out
 
 

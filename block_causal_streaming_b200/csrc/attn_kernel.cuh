@@ -16,22 +16,30 @@
 // Warp roles (384 threads):
 //   warps 0-3  softmax of Q tile 0: thread t owns query row t (TMEM lane t)
 //   warps 4-7  softmax of Q tile 1
-//   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of NS shared-memory slots,
-//              page by page through the page table; also allocates/frees TMEM
-//   warp  9    MMA issuer: S_q = Q_q K_j^T (SS form) and O_q += P_q V_j (TS form, P in TMEM)
+//   warp  8    TMA producer: Q tiles once, then K_j, V_j (BN keys each) into a ring of NS
+//              shared-memory slots, page by page through the page table; zeroes the rows of
+//              the last V tile past the last visible key; allocates/frees TMEM
+//   warp  9    MMA issuer (one thread): S_q = Q_q K_j^T (SS form) and O_q += P_q V_j (TS form,
+//              P in TMEM), in a fixed order; with two S buffers QK^T of tile j+1 goes before
+//              P.V of tile j
 //   warps 10-11 idle
-// TMEM (512 columns): S_q / P_q at columns [128q, 128q+128) (P, bf16x2, aliases the first 64),
-// O_q at [256 + D q, 256 + D q + D).
+// TMEM (512 columns): per Q tile q, NSB = 128/BN S buffers of BN fp32 columns, S_q[b] at
+// 128q + BN b (P_q of a tile, bf16x2, overwrites the first BN/2 columns of its own S buffer), and
+// O_q at 256 + Dq.  With BN = 64 the two S buffers let the softmax of tile j run while QK^T of
+// tile j+1 is computed; with BN = 128 there is one buffer and the chain is serial.
 //
 // Synchronisation (all mbarriers, all waits bounded):
-//   q_full        TMA -> MMA          Q tiles landed
-//   kv_full[s]    TMA -> MMA          K or V tile landed in slot s
-//   kv_empty[s]   MMA commit -> TMA   slot s free again (both Q tiles' MMAs on it completed)
-//   s_full[q]     MMA commit -> softmax q   S_q of tile j ready (also covers PV_q of tile j-1)
-//   p_full[q]     softmax q -> MMA    P_q of tile j written to TMEM (and O_q rescaled if needed)
-//   o_done[q]     MMA commit -> MMA / softmax   PV_q of tile j completed
-// S_q of tile j+1 overwrites the TMEM columns that PV_q of tile j reads P from, so the MMA warp
-// issues it only after o_done[q] reports that PV completed.
+//   q_full          TMA -> MMA          Q tiles landed
+//   kv_full[s]      TMA -> MMA          K or V tile landed in slot s
+//   kv_empty[s]     MMA commit -> TMA   slot s free again (both Q tiles' MMAs on it completed)
+//   s_full[q][b]    MMA commit -> softmax q   S of tile j (b = j mod NSB) ready
+//   p_full[q][b]    softmax q -> MMA    P of tile j written to TMEM (and O_q rescaled if needed)
+//   o_done[q][b]    MMA commit -> MMA / softmax   P.V of tile j (b = j mod NSB) completed
+//   v_zeroed        TMA warp -> MMA     tail rows of the last V tile zeroed
+// S of tile j+NSB overwrites the columns P.V of tile j reads P from; the PTX ordering guarantee
+// between consecutive MMAs covers only the same accumulator, so the MMA warp issues it only after
+// o_done[q][b] reports that P.V completed.  The softmax rescales O only after P.V of the
+// previous tile completed.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -41,10 +49,23 @@
 namespace wfk {
 
 constexpr int kBM = 128;        // query rows per Q tile (UMMA M)
-constexpr int kBN = 128;        // keys per K/V tile (UMMA N of QK^T, K of PV)
+#ifndef WF_ATTN_BN
+#define WF_ATTN_BN 128
+#endif
+#ifndef WF_UNIT_ORDER
+#define WF_UNIT_ORDER 0
+#endif
+#ifndef WF_KV_RING_KB
+#define WF_KV_RING_KB 128
+#endif
+constexpr int kBN = WF_ATTN_BN;  // keys per K/V tile (UMMA N of QK^T, K of PV): 64 or 128
 constexpr int kNQT = 2;         // Q tiles per CTA
 constexpr int kAttnThreads = 384;
 constexpr int kMaxQChunks = 64;
+#ifndef WF_PREFETCH_KEYS
+#define WF_PREFETCH_KEYS 0
+#endif
+constexpr int kPrefetchKeys = WF_PREFETCH_KEYS;  // L2 prefetch distance of the K/V stream (0: off)
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;   // 0.2 s when draining
 
@@ -80,29 +101,33 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-template <int D>
+template <int D, int BN>
 struct AttnSmem {
+  static constexpr int NSB = 128 / BN;                   // S buffers per Q tile
   static constexpr int DH = D / 64;                      // 128-byte halves of a row
-  static constexpr int NS = (D == 128) ? 4 : 8;          // K/V ring slots
-  static constexpr uint32_t HALF = 128u * 128u;          // 128 rows x 128 B, 128B-swizzled
-  static constexpr uint32_t TILE = DH * HALF;            // one Q, K or V tile
+  static constexpr int NS = WF_KV_RING_KB * 1024 / (int)(DH * BN * 128);   // K/V ring slots
+  static constexpr uint32_t QHALF = kBM * 128u;          // 128 rows x 128 B, 128B-swizzled
+  static constexpr uint32_t QTILE = DH * QHALF;
+  static constexpr uint32_t KHALF = BN * 128u;           // BN rows x 128 B
+  static constexpr uint32_t KTILE = DH * KHALF;          // one K or V tile
   static constexpr uint32_t Q_OFF = 0;
-  static constexpr uint32_t KV_OFF = Q_OFF + kNQT * TILE;
-  static constexpr uint32_t BAR_OFF = KV_OFF + NS * TILE;
-  // barrier indices
-  static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NS, B_S = 1 + 2 * NS, B_P = B_S + 2,
-                       B_O = B_P + 2, B_DRAIN = B_O + 2, NBAR = B_DRAIN + 1;
+  static constexpr uint32_t KV_OFF = Q_OFF + kNQT * QTILE;
+  static constexpr uint32_t BAR_OFF = KV_OFF + NS * KTILE;
+  // barrier indices; per-(q, b) barriers at base + NSB q + b
+  static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NS, B_S = 1 + 2 * NS,
+                       B_P = B_S + 2 * NSB, B_O = B_P + 2 * NSB, B_DRAIN = B_O + 2 * NSB,
+                       B_VZ = B_DRAIN + 1, NBAR = B_VZ + 1;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr uint32_t BYTES = MISC_OFF + 16;
   static constexpr uint32_t ALLOC = BYTES + 1024;        // slack for 1024-byte alignment
 };
 
-template <int D>
+template <int D, int BN>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     wf_attn_fwd_kernel(const __grid_constant__ AttnParams p) {
-  using L = AttnSmem<D>;
-  constexpr int DH = L::DH, NS = L::NS;
-  constexpr uint32_t TILE = L::TILE, HALF = L::HALF;
+  using L = AttnSmem<D, BN>;
+  constexpr int DH = L::DH, NS = L::NS, NSB = L::NSB;
+  constexpr uint32_t QTILE = L::QTILE, QHALF = L::QHALF, KTILE = L::KTILE, KHALF = L::KHALF;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -114,12 +139,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int unit = blockIdx.x;
+#if WF_UNIT_ORDER == 1
+  const int pair = p.n_pairs - 1 - unit % p.n_pairs;    // head-major: one head's K/V live at once
+  const int head = unit / p.n_pairs;
+#else
   const int pair = p.n_pairs - 1 - unit / p.H;
   const int head = unit % p.H;
+#endif
   const int m0 = pair * (kNQT * kBM);
   const int last_row = min(m0 + kNQT * kBM, p.T_q) - 1;
   const int n_max = kv_end_of_row(p, last_row);        // keys any row of this unit may see
-  const int nk = (n_max + kBN - 1) / kBN;                // K/V tiles to visit
+  const int nk = (n_max + BN - 1) / BN;                // K/V tiles to visit
 
   const WaitCtx w{cta_abort, p.grid_abort, p.status, p.launch_id, 6 /* WF_ERR_TIMEOUT */,
                   kWaitTimeoutNs};
@@ -127,7 +157,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     *cta_abort = (*reinterpret_cast<volatile unsigned*>(p.grid_abort) == p.launch_id) ? 1 : 0;
     for (int i = 0; i < L::NBAR; ++i)
-      mbar_init(bar(i), (i == L::B_P || i == L::B_P + 1) ? 128u : 1u);
+      mbar_init(bar(i), (i >= L::B_P && i < L::B_P + 2 * NSB) ? 128u : 1u);
     mbar_init_fence();
   }
   if (warp == 8) {
@@ -139,286 +169,326 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool skip = *cta_abort != 0;
+  // Registers: the kernel launches with 168 per thread (384 x 168 = 64512); the softmax
+  // warpgroups take 208 each and the producer/MMA warpgroup keeps 88
+  // (2 x 128 x 208 + 128 x 88 = 64512).  The build checks the 168.
 
-  if (!skip && warp < 8) {
-    // ------------------------------------------------------------------ softmax warpgroups
-    const int q = warp >> 2, wq = warp & 3;
-    const int row = wq * 32 + lane;                       // row within the Q tile == TMEM lane
-    const int row_g = m0 + q * kBM + row;                 // query row
-    const int n_r = kv_end_of_row(p, min(row_g, p.T_q - 1));
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + static_cast<uint32_t>(q * 128);
-    const uint32_t tO = tmem + lane_off + 256u + static_cast<uint32_t>(q * D);
-    const float sl2 = p.sl2;
-    float m2 = -INFINITY;   // running max of the base-2 logits in use
-    float l = 0.f;          // running sum of exp2(t - m2)
-    bool ok = true;
-    for (int j = 0; j < nk; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_S + q), j & 1, w));
-      if (!ok) break;
-      tc_fence_after();
-      float s[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + 32u * c, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[i]);
+  if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+    if (!skip) {
+      // ------------------------------------------------------------------ softmax warpgroups
+      const int q = warp >> 2, wq = warp & 3;
+      const int row = wq * 32 + lane;                       // row within the Q tile == TMEM lane
+      const int row_g = m0 + q * kBM + row;                 // query row
+      const int n_r = kv_end_of_row(p, min(row_g, p.T_q - 1));
+      const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+      const uint32_t tS0 = tmem + lane_off + static_cast<uint32_t>(q * 128);
+      const uint32_t tO = tmem + lane_off + 256u + static_cast<uint32_t>(q * D);
+      const float sl2 = p.sl2;
+      float m2 = -INFINITY;   // running max of the base-2 logits in use
+      float l = 0.f;          // running sum of exp2(t - m2)
+      bool ok = true;
+      const float2 sl2x2 = make_float2(sl2, sl2);
+      for (int j = 0; j < nk; ++j) {
+        const int b = j % NSB;
+        const uint32_t tS = tS0 + static_cast<uint32_t>(BN * b);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_S + NSB * q + b), (j / NSB) & 1, w));
+        if (!ok) break;
+        tc_fence_after();
+        float s[BN];
+        {
+          uint32_t r[BN];
+  #pragma unroll
+          for (int c = 0; c < BN / 32; ++c)
+            tmem_ld32(tS + 32u * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+          tmem_wait_ld();
+  #pragma unroll
+          for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
+        }
+        const int lim = n_r - j * BN;                       // visible columns of this tile
+        const bool masked = lim < BN;
+        if (masked) {
+  #pragma unroll
+          for (int c = 0; c < BN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+        }
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+  #pragma unroll
+        for (int c = 4; c < BN; c += 8) {
+          mx0 = max3(mx0, s[c], s[c + 1]);
+          mx1 = max3(mx1, s[c + 2], s[c + 3]);
+          if (c + 4 < BN) mx2 = max3(mx2, s[c + 4], s[c + 5]);
+          if (c + 6 < BN) mx3 = max3(mx3, s[c + 6], s[c + 7]);
+        }
+        const float tmax = max3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
+        // Move the reference max only when the new one exceeds it by more than 2^8: O and l both
+        // stay expressed against the same stale reference, so O / l is unchanged, and every
+        // exp2(t - m2) stays <= 256.
+        const bool need = tmax > m2 + 8.0f;
+        float alpha = 1.f;
+        if (need) {
+          alpha = ex2_approx(m2 - tmax);                   // 0 on the first visible tile
+          m2 = tmax;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O_q holds P.V of tiles < j once P.V of tile j-1 has completed; rescale this warp's
+          // rows (threads whose max did not move multiply by 1).
+          const int bp = (j - 1) % NSB;
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(bar(L::B_O + NSB * q + bp), ((j - 1) / NSB) & 1, w));
+          if (!ok) break;
+          tc_fence_after();
+  #pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + 32u * c, r);
+            tmem_wait_ld();
+  #pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(tO + 32u * c, r);
+          }
+        }
+        l *= alpha;
+        // p = exp2(s * scale * log2 e - m2) two columns at a time.  On unmasked tiles 3 of every
+        // 8 column pairs use the FMA-pipe polynomial and the rest the MUFU unit, which alone
+        // would be as slow as the tensor core at head_dim 128.  Masked tiles use the MUFU unit
+        // only, so masked columns give exactly 0.
+        const float2 negm = make_float2(-m2, -m2);
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        uint32_t pk[BN / 2];
+        if (!masked) {
+  #pragma unroll
+          for (int i = 0; i < BN / 2; ++i) {
+            const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2x2, negm);
+            float2 e;
+            if ((i & 7) < 3) {
+              e = exp2_poly2(x);
+            } else {
+              e.x = ex2_approx(x.x);
+              e.y = ex2_approx(x.y);
+            }
+            if (i & 1) acc1 = __fadd2_rn(acc1, e); else acc0 = __fadd2_rn(acc0, e);
+            pk[i] = pack_bf16x2(e.x, e.y);
+          }
+        } else {
+  #pragma unroll
+          for (int i = 0; i < BN / 2; ++i) {
+            const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2x2, negm);
+            const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (i & 1) acc1 = __fadd2_rn(acc1, e); else acc0 = __fadd2_rn(acc0, e);
+            pk[i] = pack_bf16x2(e.x, e.y);
+          }
+        }
+  #pragma unroll
+        for (int h = 0; h < BN / 64; ++h)
+          tmem_st32(tS + 32u * h, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h]));
+        const float2 acc = __fadd2_rn(acc0, acc1);
+        l += acc.x + acc.y;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::B_P + NSB * q + b));
       }
-      const int lim = n_r - j * kBN;                      // visible columns of this tile
-      if (lim < kBN) {
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
-      }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-      for (int c = 4; c < kBN; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
-      }
-      const float tmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-      // Move the reference max only when the new one exceeds it by more than 2^8: O and l both
-      // stay expressed against the same stale reference, so O / l is unchanged, and every
-      // exp2(t - m2) stays <= 256.
-      const bool need = tmax > m2 + 8.0f;
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2_approx(m2 - tmax);                   // 0 on the first visible tile
-        m2 = tmax;
-      }
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // O_q holds PV of tiles < j (the s_full commit covered it); rescale this warp's rows.
-#pragma unroll
+      // ------------------------------------------------------------------------- epilogue
+      if (ok)
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(bar(L::B_O + NSB * q + (nk - 1) % NSB), ((nk - 1) / NSB) & 1, w));
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        const bool live = row_g < p.T_q;
+        __nv_bfloat16* const orow = p.out + (static_cast<size_t>(row_g) * p.H + head) * D;
+  #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
           tmem_ld32(tO + 32u * c, r);
           tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(tO + 32u * c, r);
+          if (live) {
+            uint32_t pk[16];
+  #pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l,
+                                  __uint_as_float(r[2 * i + 1]) * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+  #pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
         }
+        if (p.lse != nullptr && live)
+          p.lse[static_cast<size_t>(head) * p.T_q + row_g] = (m2 + __log2f(l)) * 0.69314718056f;
       }
-      l *= alpha;
-      const float negm = -m2;
-      float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(s[64 * h + 2 * i], sl2, negm));
-          const float p1 = ex2_approx(fmaf(s[64 * h + 2 * i + 1], sl2, negm));
-          rs0 += p0;
-          rs1 += p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + 32u * h, pk);
+    }
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+    if (!skip && warp == 8) {
+      // ------------------------------------------------------------------------ TMA producer
+      const int R = p.box_rows, nb = BN / R;             // page boxes per K/V tile (<= BN/16)
+      bool ok = true;
+      int last_it[NS];
+  #pragma unroll
+      for (int s = 0; s < NS; ++s) last_it[s] = -1;
+      if (lane == 0) {
+        tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_k);
+        tma_prefetch_desc(&p.tm_v);
+        mbar_arrive_expect_tx(bar(L::B_Q), kNQT * QTILE);
+  #pragma unroll
+        for (int qt = 0; qt < kNQT; ++qt)
+  #pragma unroll
+          for (int h = 0; h < DH; ++h)
+            tma_load_3d(base + L::Q_OFF + qt * QTILE + h * QHALF, &p.tm_q, 64 * h, head,
+                        m0 + qt * kBM, bar(L::B_Q));
       }
-      l += rs0 + rs1;
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(L::B_P + q));
-    }
-    // ------------------------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_O + q), (nk - 1) & 1, w));
-    if (ok) {
-      tc_fence_after();
-      const float inv_l = 1.f / l;
-      const bool live = row_g < p.T_q;
-      __nv_bfloat16* const orow = p.out + (static_cast<size_t>(row_g) * p.H + head) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + 32u * c, r);
-        tmem_wait_ld();
-        if (live) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l,
-                                __uint_as_float(r[2 * i + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-        }
-      }
-      if (p.lse != nullptr && live)
-        p.lse[static_cast<size_t>(head) * p.T_q + row_g] = (m2 + __log2f(l)) * 0.69314718056f;
-    }
-  } else if (!skip && warp == 8) {
-    // ------------------------------------------------------------------------ TMA producer
-    const int R = p.box_rows, nb = kBN / R;             // page boxes per K/V tile (<= 8)
-    bool ok = true;
-    int last_it[NS];
-#pragma unroll
-    for (int s = 0; s < NS; ++s) last_it[s] = -1;
-    if (lane == 0) {
-      tma_prefetch_desc(&p.tm_q);
-      tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_v);
-      mbar_arrive_expect_tx(bar(L::B_Q), kNQT * TILE);
-#pragma unroll
-      for (int qt = 0; qt < kNQT; ++qt)
-#pragma unroll
-        for (int h = 0; h < DH; ++h)
-          tma_load_3d(base + L::Q_OFF + qt * TILE + h * HALF, &p.tm_q, 64 * h, head,
-                      m0 + qt * kBM, bar(L::B_Q));
-    }
-    for (int j = 0; j < nk && ok; ++j) {
-      // lane b resolves the physical row of box b of this tile
-      int coord = p.total_rows;                          // past the pool: TMA fills zeros
-      const int tok = j * kBN + lane * R;
-      if (lane < nb && tok < n_max) {
+      // Physical row of box b of tile t (past the pool -- TMA fills zeros -- beyond n_max).
+      auto box_row = [&](int t, int b) -> int {
+        const int tok = t * BN + b * R;
+        if (b >= nb || t >= nk || tok >= n_max) return p.total_rows;
         int pg = __ldg(p.page_table + tok / p.page_size);
         if (pg < 0 || pg >= p.num_pages) {
           atomicCAS(p.status, 0, 5 /* WF_ERR_PAGE_OOB */);
           pg = 0;
         }
-        coord = pg * p.page_size + tok % p.page_size;
-      }
-      int cb[8];
-#pragma unroll
-      for (int b = 0; b < 8; ++b) cb[b] = __shfl_sync(0xffffffffu, coord, b);
-      if (lane == 0) {
-#pragma unroll
-        for (int kv = 0; kv < 2 && ok; ++kv) {
-          const int it = 2 * j + kv, slot = it % NS;
-          ok = mbar_wait(bar(L::B_KVE + slot), ((it / NS) & 1) ^ 1, w);
-          if (!ok) break;
-          mbar_arrive_expect_tx(bar(L::B_KVF + slot), TILE);
-          const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
-          const uint32_t dst = base + L::KV_OFF + slot * TILE;
-#pragma unroll
-          for (int b = 0; b < 8; ++b) {
-            if (b < nb) {
-#pragma unroll
-              for (int h = 0; h < DH; ++h)
-                tma_load_3d(dst + h * HALF + static_cast<uint32_t>(b * R * 128), map, 64 * h,
-                            head, cb[b], bar(L::B_KVF + slot));
-            }
-          }
-          last_it[slot] = it;
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-    }
-    if (lane == 0) {
-      // every load this warp issued must land before shared memory is released
-      mbar_wait_drain(bar(L::B_Q), 0);
-#pragma unroll
-      for (int s = 0; s < NS; ++s)
-        if (last_it[s] >= 0) mbar_wait_drain(bar(L::B_KVF + s), (last_it[s] / NS) & 1);
-    }
-  } else if (!skip && warp == 9) {
-    // ---------------------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);   // Q, K both K-major
-    constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);     // P (TMEM), V MN-major
-    bool ok = true;
-    if (lane == 0) ok = mbar_wait(bar(L::B_Q), 0, w);
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    int js[2] = {0, 0};   // next tile whose S is to be issued, per Q tile
-    int jp[2] = {0, 0};   // next tile whose PV is to be issued, per Q tile
-    bool vz_done = false;
-    const int zero_from = n_max - (nk - 1) * kBN;         // rows >= this of the last V tile
-    uint64_t t_last = globaltimer_ns();
-    unsigned idle = 0;
-    while (ok && (jp[0] < nk || jp[1] < nk)) {
-      int action = -1;   // 0/1: S of Q tile 0/1;  2/3: PV of Q tile 0/1
-      if (lane == 0) {
-#pragma unroll
-        for (int q = 0; q < 2 && action < 0; ++q) {
-          const int j = js[q];
-          if (j < nk && j == jp[q]) {
-            const int it = 2 * j;
-            if (mbar_test(bar(L::B_KVF + it % NS), (it / NS) & 1) &&
-                (j == 0 || mbar_test(bar(L::B_O + q), (j - 1) & 1)))
-              action = q;
+        return pg * p.page_size + tok % p.page_size;
+      };
+      // Tiles are also prefetched into L2 kPrefetchKeys ahead: every CTA of a head streams the
+      // same K/V at about the same time, so without it each tile would wait on an HBM round trip.
+      constexpr int PF = kPrefetchKeys / BN;
+      auto prefetch_tile = [&](int t, int row) {            // row: this lane's box row of tile t
+        if (PF > 0 && lane < nb && row < p.total_rows) {
+  #pragma unroll
+          for (int h = 0; h < DH; ++h) {
+            tma_prefetch_l2_3d(&p.tm_k, 64 * h, head, row);
+            tma_prefetch_l2_3d(&p.tm_v, 64 * h, head, row);
           }
         }
-#pragma unroll
-        for (int q = 0; q < 2 && action < 0; ++q) {
-          const int j = jp[q];
-          if (j < js[q]) {
-            const int it = 2 * j + 1;
-            if (mbar_test(bar(L::B_P + q), j & 1) &&
-                mbar_test(bar(L::B_KVF + it % NS), (it / NS) & 1))
-              action = 2 + q;
-          }
-        }
-        if (action < 0) {
-          if ((++idle & 255u) == 0) {
-            if (aborted(w)) {
-              ok = false;
-            } else if (globaltimer_ns() - t_last > kWaitTimeoutNs) {
-              raise_abort(w);
-              ok = false;
-            }
-          }
-        } else {
-          idle = 0;
-          t_last = globaltimer_ns();
-        }
-      }
-      action = __shfl_sync(0xffffffffu, action, 0);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (action < 0) continue;
-      if (action < 2) {
-        const int q = action, j = js[q], it = 2 * j, slot = it % NS;
+      };
+      for (int t = 1; t < PF && t < nk; ++t) prefetch_tile(t, box_row(t, lane));
+      (void)prefetch_tile;
+      for (int j = 0; j < nk && ok; ++j) {
+        const int coord = box_row(j, lane);                 // lane b resolves box b of tile j
+        if (PF > 0) prefetch_tile(j + PF, box_row(j + PF, lane));
+        int cb[BN / 16];
+  #pragma unroll
+        for (int b = 0; b < BN / 16; ++b) cb[b] = __shfl_sync(0xffffffffu, coord, b);
         if (lane == 0) {
-          tc_fence_after();
-          const uint32_t qa = base + L::Q_OFF + q * TILE;
-          const uint32_t kb = base + L::KV_OFF + slot * TILE;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk / 4) * HALF + (kk % 4) * 32;   // 16 bf16 = 32 B per step
-            umma_ss(tmem + static_cast<uint32_t>(q * 128), smem_desc_sw128(qa + off, 16, 1024),
-                    smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+  #pragma unroll
+          for (int kv = 0; kv < 2 && ok; ++kv) {
+            const int it = 2 * j + kv, slot = it % NS;
+            ok = mbar_wait(bar(L::B_KVE + slot), ((it / NS) & 1) ^ 1, w);
+            if (!ok) break;
+            mbar_arrive_expect_tx(bar(L::B_KVF + slot), KTILE);
+            const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
+            const uint32_t dst = base + L::KV_OFF + slot * KTILE;
+  #pragma unroll
+            for (int b = 0; b < BN / 16; ++b) {
+              if (b < nb) {
+  #pragma unroll
+                for (int h = 0; h < DH; ++h)
+                  tma_load_3d(dst + h * KHALF + static_cast<uint32_t>(b * R * 128), map, 64 * h,
+                              head, cb[b], bar(L::B_KVF + slot));
+              }
+            }
+            last_it[slot] = it;
           }
-          umma_commit(bar(L::B_S + q));
-          if (js[1 - q] > j) umma_commit(bar(L::B_KVE + slot));     // both Q tiles done with K_j
         }
-        js[q] = j + 1;
-      } else {
-        const int q = action - 2, j = jp[q], it = 2 * j + 1, slot = it % NS;
-        const uint32_t vb = base + L::KV_OFF + slot * TILE;
-        if (j == nk - 1 && zero_from < kBN && !vz_done) {
-          // Rows past the last visible key may hold anything (even NaN, which 0 * NaN would
-          // spread); zero them before any PV reads this tile.
-          __syncwarp();
-          const int n16 = (kBN - zero_from) * 8;                 // 16-byte pieces per half
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+      const int zero_from = n_max - (nk - 1) * BN;         // rows >= this of the last V tile
+      if (ok && zero_from < BN) {
+        // Rows past the last visible key may hold anything (even NaN, which 0 * NaN would spread
+        // through P.V); once the last V tile has landed, zero them and release the MMA warp.
+        const int it = 2 * (nk - 1) + 1, slot = it % NS;
+        if (lane == 0) ok = mbar_wait(bar(L::B_KVF + slot), (it / NS) & 1, w);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok) {
+          const uint32_t vb = base + L::KV_OFF + slot * KTILE;
+          const int n16 = (BN - zero_from) * 8;            // 16-byte pieces per 128-byte half
           for (int i = lane; i < n16 * DH; i += 32) {
             const int h = i / n16, rr = i % n16;
-            const uint32_t a = vb + h * HALF + static_cast<uint32_t>(zero_from * 128 + rr * 16);
+            const uint32_t a = vb + h * KHALF + static_cast<uint32_t>(zero_from * 128 + rr * 16);
             asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
           }
           fence_proxy_async_smem();
           __syncwarp();
-          vz_done = true;
+          if (lane == 0) mbar_arrive(bar(L::B_VZ));
         }
-        if (lane == 0) {
-          tc_fence_after();
-          const uint32_t pa = tmem + static_cast<uint32_t>(q * 128);
-          const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_ts(od, pa + 8u * kk, smem_desc_sw128(vb + kk * 2048u, HALF, 1024), idesc_pv,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(bar(L::B_O + q));
-          if (jp[1 - q] > j) umma_commit(bar(L::B_KVE + slot));     // both Q tiles done with V_j
-        }
-        jp[q] = j + 1;
       }
-    }
-    if (lane == 0) {
-      // every MMA this warp issued must complete before TMEM is released
+      if (lane == 0) {
+        // every load this warp issued must land before shared memory is released
+        mbar_wait_drain(bar(L::B_Q), 0);
+  #pragma unroll
+        for (int s = 0; s < NS; ++s)
+          if (last_it[s] >= 0) mbar_wait_drain(bar(L::B_KVF + s), (last_it[s] / NS) & 1);
+      }
+    } else if (!skip && warp == 9 && lane == 0) {
+      // ---------------------------------------------------------------------- MMA issuer
+      // One thread issues everything in a fixed order.  Descriptors are built once; per
+      // instruction only a compile-time offset (16-byte units) is added to the start-address
+      // field, so one MMA costs a few instructions to issue -- the tensor core retires a
+      // 128 x BN x 16 step in BN/2 cycles and must not wait for the issuer.
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, BN, 0, 0);   // Q, K both K-major
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);     // P (TMEM), V MN-major
+      const uint64_t dq0 = smem_desc_sw128(base + L::Q_OFF, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(base + L::KV_OFF, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(base + L::KV_OFF, KHALF, 1024);
+      const bool zero_tail = (n_max - (nk - 1) * BN) < BN;   // the loader zeroes V's tail rows
+      bool ok = mbar_wait(bar(L::B_Q), 0, w);
+
+      // S_q(j) = Q_q K_j^T into S buffer j mod NSB, once P.V of tile j-NSB has released it.
+      auto issue_s = [&](int j) -> bool {
+        const int it = 2 * j, slot = it % NS;
+        if (!mbar_wait(bar(L::B_KVF + slot), (it / NS) & 1, w)) return false;
+        const uint64_t dk = dk0 + ((static_cast<uint32_t>(slot) * KTILE) >> 4);
+  #pragma unroll
+        for (int q = 0; q < kNQT; ++q) {
+          if (j >= NSB &&
+              !mbar_wait(bar(L::B_O + NSB * q + j % NSB), ((j - NSB) / NSB) & 1, w))
+            return false;
+          tc_fence_after();
+          const uint32_t sd = tmem + static_cast<uint32_t>(q * 128 + BN * (j % NSB));
+          const uint64_t dq = dq0 + ((static_cast<uint32_t>(q) * QTILE) >> 4);
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)   // 16 bf16 = 32 B per K-step; 64 per 128-B half
+            umma_ss(sd, dq + (((kk / 4) * QHALF + (kk % 4) * 32) >> 4),
+                    dk + (((kk / 4) * KHALF + (kk % 4) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+          umma_commit(bar(L::B_S + NSB * q + j % NSB));
+        }
+        umma_commit(bar(L::B_KVE + slot));          // K_j free once both Q tiles' MMAs finish
+        return true;
+      };
+      // O_q += P_q(j) V_j, P read from TMEM (the first BN/2 columns of S buffer j mod NSB).
+      auto issue_pv = [&](int j) -> bool {
+        const int it = 2 * j + 1, slot = it % NS;
+        if (!mbar_wait(bar(L::B_KVF + slot), (it / NS) & 1, w)) return false;
+        if (j == nk - 1 && zero_tail && !mbar_wait(bar(L::B_VZ), 0, w)) return false;
+        const uint64_t dv = dv0 + ((static_cast<uint32_t>(slot) * KTILE) >> 4);
+  #pragma unroll
+        for (int q = 0; q < kNQT; ++q) {
+          if (!mbar_wait(bar(L::B_P + NSB * q + j % NSB), (j / NSB) & 1, w)) return false;
+          tc_fence_after();
+          const uint32_t pa = tmem + static_cast<uint32_t>(q * 128 + BN * (j % NSB));
+          const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
+  #pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)      // 16 keys = 8 TMEM columns / 2 KB of V
+            umma_ts(od, pa + 8u * kk, dv + ((kk * 2048u) >> 4), idesc_pv,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar(L::B_O + NSB * q + j % NSB));
+        }
+        umma_commit(bar(L::B_KVE + slot));          // V_j free once both P.V finish
+        return true;
+      };
+
+      // With two S buffers, QK^T of tile j+1 is issued before P.V of tile j so the tensor pipe
+      // has work while the softmax of tile j runs.
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < nk; ++j) {
+        if (NSB > 1 && j + 1 < nk) ok = issue_s(j + 1);
+        if (ok) ok = issue_pv(j);
+        if (NSB == 1 && ok && j + 1 < nk) ok = issue_s(j + 1);
+      }
+      // every MMA this thread issued must complete before TMEM is released
       umma_commit(bar(L::B_DRAIN));
       mbar_wait_drain(bar(L::B_DRAIN), 0);
     }
-    __syncwarp();
   }
 
   tc_fence_before();

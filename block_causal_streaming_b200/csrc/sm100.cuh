@@ -90,15 +90,23 @@ __device__ __forceinline__ void raise_abort(const WaitCtx& w) {
   __threadfence();
 }
 
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, WaitCtx w) {
+static __device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, WaitCtx w) {
   const uint64_t t0 = globaltimer_ns();
-  for (;;) {
-    for (int i = 0; i < 16; ++i)
-      if (mbar_try(bar, parity)) return true;
-    if (aborted(w)) return false;
-    if (globaltimer_ns() - t0 > w.timeout_ns) {
-      raise_abort(w);
-      return false;
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    // The abort words and the clock are consulted rarely: the grid-wide word is an uncached
+    // global load, which would otherwise delay every wake-up by an L2 round trip.
+    if ((i & 255u) == 0) {
+      if (*w.cta_abort != 0) return false;
+      if (globaltimer_ns() - t0 > w.timeout_ns) {
+        raise_abort(w);
+        return false;
+      }
+      if ((i & 4095u) == 0 &&
+          *reinterpret_cast<volatile unsigned*>(w.grid_abort) == w.launch_id) {
+        *w.cta_abort = 1;
+        return false;
+      }
     }
   }
 }
@@ -120,6 +128,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const CUtensorMap
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
       : "memory");
+}
+
+// 3-D tiled prefetch global -> L2 only (no shared memory written, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
@@ -256,6 +272,38 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Coefficients of a degree-3 polynomial for 2^f on [-1/2, 1/2], fitted for minimal maximum
+// relative error (Lawson's iteratively reweighted least squares on Chebyshev nodes; see
+// exp2_poly.py beside this file).  Maximum relative error 7.5e-5, evaluated in fp32.
+constexpr float kExp2C0 = 0.99992805719375610f;
+constexpr float kExp2C1 = 0.69326096773147583f;
+constexpr float kExp2C2 = 0.24261112511157990f;
+constexpr float kExp2C3 = 0.05517166480422020f;
+
+// 2^x for two values on the FMA pipe instead of the MUFU unit (Cody-Waite style split):
+// x is clamped to >= -126, n = round(x) is formed by adding 1.5 * 2^23 (so n sits in the low
+// mantissa bits), f = x - n lies in [-1/2, 1/2], 2^f comes from the polynomial above, and 2^n is
+// added to the exponent field.  For x >= -126 the exponent never leaves the normal range; below
+// that the result is a tiny positive number instead of the exact underflow to 0.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
+  p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 }  // namespace wfk

@@ -59,12 +59,12 @@ int device_state(DeviceState** out) {
         if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_wf_status) != cudaSuccess ||
             cudaGetSymbolAddress(reinterpret_cast<void**>(&d.abort_word), g_wf_abort) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<128>,
+            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<128, wfk::kBN>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 wfk::AttnSmem<128>::ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<64>,
+                                 wfk::AttnSmem<128, wfk::kBN>::ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<64, wfk::kBN>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 wfk::AttnSmem<64>::ALLOC) != cudaSuccess) {
+                                 wfk::AttnSmem<64, wfk::kBN>::ALLOC) != cudaSuccess) {
           cudaGetLastError();
           return WF_ERR_CUDA;
         }
@@ -264,11 +264,11 @@ int wf_attn_forward(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* 
   if (grid > INT32_MAX) return WF_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (D == 128)
-    wfk::wf_attn_fwd_kernel<128><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
-                                   wfk::AttnSmem<128>::ALLOC, s>>>(p);
+    wfk::wf_attn_fwd_kernel<128, wfk::kBN><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
+                                             wfk::AttnSmem<128, wfk::kBN>::ALLOC, s>>>(p);
   else
-    wfk::wf_attn_fwd_kernel<64><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
-                                  wfk::AttnSmem<64>::ALLOC, s>>>(p);
+    wfk::wf_attn_fwd_kernel<64, wfk::kBN><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
+                                            wfk::AttnSmem<64, wfk::kBN>::ALLOC, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
