@@ -52,6 +52,12 @@ constexpr int kBM = 128;        // query rows per Q tile (UMMA M)
 #ifndef WF_ATTN_BN
 #define WF_ATTN_BN 128
 #endif
+#ifndef WF_EXP2_POLY_EIGHTHS
+#define WF_EXP2_POLY_EIGHTHS 2   // column pairs out of 8 whose exp2 runs on the FMA pipe
+#endif
+#ifndef WF_SOFTMAX_PINGPONG
+#define WF_SOFTMAX_PINGPONG 0     // 1: the two softmax warpgroups take turns on the exp phase
+#endif
 #ifndef WF_UNIT_ORDER
 #define WF_UNIT_ORDER 0
 #endif
@@ -116,7 +122,7 @@ struct AttnSmem {
   // barrier indices; per-(q, b) barriers at base + NSB q + b
   static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NS, B_S = 1 + 2 * NS,
                        B_P = B_S + 2 * NSB, B_O = B_P + 2 * NSB, B_DRAIN = B_O + 2 * NSB,
-                       B_VZ = B_DRAIN + 1, NBAR = B_VZ + 1;
+                       B_VZ = B_DRAIN + 1, B_TOK = B_VZ + 1, NBAR = B_TOK + 2;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr uint32_t BYTES = MISC_OFF + 16;
   static constexpr uint32_t ALLOC = BYTES + 1024;        // slack for 1024-byte alignment
@@ -157,7 +163,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     *cta_abort = (*reinterpret_cast<volatile unsigned*>(p.grid_abort) == p.launch_id) ? 1 : 0;
     for (int i = 0; i < L::NBAR; ++i)
-      mbar_init(bar(i), (i >= L::B_P && i < L::B_P + 2 * NSB) ? 128u : 1u);
+      mbar_init(bar(i), ((i >= L::B_P && i < L::B_P + 2 * NSB) || i >= L::B_TOK) ? 128u : 1u);
     mbar_init_fence();
   }
   if (warp == 8) {
@@ -189,6 +195,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float l = 0.f;          // running sum of exp2(t - m2)
       bool ok = true;
       const float2 sl2x2 = make_float2(sl2, sl2);
+      if (WF_SOFTMAX_PINGPONG && q == 1) mbar_arrive(bar(L::B_TOK + 0));   // warpgroup 0 goes first
       for (int j = 0; j < nk; ++j) {
         const int b = j % NSB;
         const uint32_t tS = tS0 + static_cast<uint32_t>(BN * b);
@@ -252,6 +259,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // 8 column pairs use the FMA-pipe polynomial and the rest the MUFU unit, which alone
         // would be as slow as the tensor core at head_dim 128.  Masked tiles use the MUFU unit
         // only, so masked columns give exactly 0.
+        if (WF_SOFTMAX_PINGPONG) {
+          // take turns with the other Q tile's warpgroup on the exp phase (token j of this one)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_TOK + q), j & 1, w));
+          if (!ok) break;
+        }
         const float2 negm = make_float2(-m2, -m2);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         uint32_t pk[BN / 2];
@@ -260,7 +272,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int i = 0; i < BN / 2; ++i) {
             const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2x2, negm);
             float2 e;
-            if ((i & 7) < 3) {
+            if ((i & 7) < WF_EXP2_POLY_EIGHTHS) {
               e = exp2_poly2(x);
             } else {
               e.x = ex2_approx(x.x);
@@ -281,6 +293,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   #pragma unroll
         for (int h = 0; h < BN / 64; ++h)
           tmem_st32(tS + 32u * h, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h]));
+        if (WF_SOFTMAX_PINGPONG) mbar_arrive(bar(L::B_TOK + 1 - q));
         const float2 acc = __fadd2_rn(acc0, acc1);
         l += acc.x + acc.y;
         tmem_wait_st();
