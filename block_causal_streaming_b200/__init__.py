@@ -14,6 +14,7 @@ _ABI_NAMES = (
     "WF_OK", "WF_ERR_INVALID_ARG", "WF_ERR_SHAPE", "WF_ERR_STAGE_ORDER", "WF_ERR_CAPACITY",
     "WF_ERR_PAGE_OOB", "WF_ERR_TIMEOUT", "WF_ERR_CUDA", "WF_ERR_NO_DEVICE", "WF_MAX_CHUNKS",
     "WavefrontDesc", "WfError", "attn_forward", "check_status", "kv_append", "strerror",
+    "selftest_timeout",
 )
 __all__ = list(_ABI_NAMES)
 

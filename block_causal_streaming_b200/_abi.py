@@ -25,7 +25,8 @@ WF_ERR_NO_DEVICE = 8
 WF_MAX_CHUNKS = 64
 
 # Every symbol include/wf.h declares (checked by the CPU tests).
-EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror", "wf_version")
+EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror", "wf_version",
+            "wf_selftest_timeout")
 
 
 class WfError(RuntimeError):
@@ -66,6 +67,8 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wf_strerror.restype = ctypes.c_char_p
     lib.wf_version.argtypes = []
     lib.wf_version.restype = i32
+    lib.wf_selftest_timeout.argtypes = [ctypes.c_uint, vp]
+    lib.wf_selftest_timeout.restype = i32
     return lib
 
 
@@ -150,6 +153,13 @@ def attn_forward(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: fl
         _stream_handle(stream))
     if rc != WF_OK:
         raise WfError(rc, "wf_attn_forward")
+
+
+def selftest_timeout(timeout_us: int, stream=None) -> None:
+    """wf_selftest_timeout: make one bounded in-kernel wait run out (read it with check_status)."""
+    rc = lib.wf_selftest_timeout(int(timeout_us), _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_selftest_timeout")
 
 
 def check_status(stream=None) -> int:

@@ -55,6 +55,9 @@ constexpr int kBM = 128;        // query rows per Q tile (UMMA M)
 #ifndef WF_EXP2_POLY_EIGHTHS
 #define WF_EXP2_POLY_EIGHTHS 2   // column pairs out of 8 whose exp2 runs on the FMA pipe
 #endif
+#ifndef WF_MMA_ORDER
+#define WF_MMA_ORDER 0   // 1: staggered Q tiles, QK^T issued as two 64-key halves, P in columns 64..127
+#endif
 #ifndef WF_SOFTMAX_PINGPONG
 #define WF_SOFTMAX_PINGPONG 0     // 1: the two softmax warpgroups take turns on the exp phase
 #endif
@@ -66,8 +69,23 @@ constexpr int kBM = 128;        // query rows per Q tile (UMMA M)
 #endif
 constexpr int kBN = WF_ATTN_BN;  // keys per K/V tile (UMMA N of QK^T, K of PV): 64 or 128
 constexpr int kNQT = 2;         // Q tiles per CTA
+constexpr uint32_t kPCol = WF_MMA_ORDER == 1 ? 64u : 0u;   // TMEM column of P within its S buffer
 constexpr int kAttnThreads = 384;
+#ifndef WF_REG_SOFTMAX
+#define WF_REG_SOFTMAX 208
+#endif
+// Register split: the kernel launches with 168 per thread (384 x 168 = 64512); the two softmax
+// warpgroups take kRegSoftmax each and the producer/MMA warpgroup keeps the rest.
+constexpr int kRegSoftmax = WF_REG_SOFTMAX;
+constexpr int kRegOther = 3 * 168 - 2 * kRegSoftmax;
+static_assert(kRegSoftmax % 8 == 0 && kRegOther % 8 == 0 && kRegOther >= 24,
+              "setmaxnreg counts are multiples of 8");
+static_assert(2 * 128 * kRegSoftmax + 128 * kRegOther <= 384 * 168, "split exceeds the launch");
 constexpr int kMaxQChunks = 64;
+#ifndef WF_PT_CACHE
+#define WF_PT_CACHE 0      // 0: each tile reads its page-table entries from global memory
+#endif
+constexpr int kPtCache = WF_PT_CACHE;   // page-table entries a producer keeps in shared memory
 #ifndef WF_PREFETCH_KEYS
 #define WF_PREFETCH_KEYS 0
 #endif
@@ -85,6 +103,7 @@ struct AttnParams {
   int* status;
   unsigned* grid_abort;
   int T_q, H, num_pages, page_size, total_rows, box_rows, n_pairs;
+  int box_rows_v;     // V box rows (CTA-pair kernel: V half-tiles of 128 keys)
   float sl2;  // scale * log2(e)
   unsigned launch_id;
   int nqc;                          // non-empty query chunks
@@ -96,6 +115,31 @@ __device__ __forceinline__ int kv_end_of_row(const AttnParams& p, int r) {
   for (int c = 0; c < p.nqc; ++c)
     if (r < p.qc_row_end[c]) return p.qc_kv_end[c];
   return p.qc_kv_end[p.nqc - 1];
+}
+
+// The producer warp copies the page-table entries of the unit's key range into shared memory
+// once (up to kPtCache of them), so each K/V tile costs a shared-memory read instead of a
+// dependent global load.  Returns the number of cached entries.
+__device__ __forceinline__ int cache_page_table(const AttnParams& p, int* pt_s, int n_max,
+                                                int lane) {
+  const int pages = (n_max + p.page_size - 1) / p.page_size;
+  const int n = min(pages, kPtCache);
+  for (int i = lane; i < n; i += 32) pt_s[i] = __ldg(p.page_table + i);
+  __syncwarp();
+  return n;
+}
+
+// Physical pool row of logical token `tok` (< n_max); entries outside the pool are recorded
+// as WF_ERR_PAGE_OOB and read as page 0.
+__device__ __forceinline__ int pool_row(const AttnParams& p, const int* pt_s, int n_cached,
+                                        int tok) {
+  const int idx = tok / p.page_size;
+  int pg = idx < n_cached ? pt_s[idx] : __ldg(p.page_table + idx);
+  if (pg < 0 || pg >= p.num_pages) {
+    atomicCAS(p.status, 0, 5 /* WF_ERR_PAGE_OOB */);
+    pg = 0;
+  }
+  return pg * p.page_size + (tok - idx * p.page_size);
 }
 
 // Wait on a phase with only a timeout (no abort check): used to drain in-flight async work
@@ -123,7 +167,8 @@ struct AttnSmem {
   static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NS, B_S = 1 + 2 * NS,
                        B_P = B_S + 2 * NSB, B_O = B_P + 2 * NSB, B_DRAIN = B_O + 2 * NSB,
                        B_VZ = B_DRAIN + 1, B_TOK = B_VZ + 1, NBAR = B_TOK + 2;
-  static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr uint32_t PT_OFF = BAR_OFF + NBAR * 8;   // page-table cache
+  static constexpr uint32_t MISC_OFF = PT_OFF + kPtCache * 4;
   static constexpr uint32_t BYTES = MISC_OFF + 16;
   static constexpr uint32_t ALLOC = BYTES + 1024;        // slack for 1024-byte alignment
 };
@@ -163,7 +208,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     *cta_abort = (*reinterpret_cast<volatile unsigned*>(p.grid_abort) == p.launch_id) ? 1 : 0;
     for (int i = 0; i < L::NBAR; ++i)
-      mbar_init(bar(i), ((i >= L::B_P && i < L::B_P + 2 * NSB) || i >= L::B_TOK) ? 128u : 1u);
+      mbar_init(bar(i), ((i >= L::B_P && i < L::B_O) || i >= L::B_TOK) ? 128u : 1u);
     mbar_init_fence();
   }
   if (warp == 8) {
@@ -175,12 +220,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool skip = *cta_abort != 0;
-  // Registers: the kernel launches with 168 per thread (384 x 168 = 64512); the softmax
-  // warpgroups take 208 each and the producer/MMA warpgroup keeps 88
-  // (2 x 128 x 208 + 128 x 88 = 64512).  The build checks the 168.
+  // Registers: see kRegSoftmax; the build checks the 168 the split relies on.
 
   if (warp < 8) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax) : "memory");
     if (!skip) {
       // ------------------------------------------------------------------ softmax warpgroups
       const int q = warp >> 2, wq = warp & 3;
@@ -292,7 +335,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
   #pragma unroll
         for (int h = 0; h < BN / 64; ++h)
-          tmem_st32(tS + 32u * h, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h]));
+          tmem_st32(tS + kPCol + 32u * h, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h]));
         if (WF_SOFTMAX_PINGPONG) mbar_arrive(bar(L::B_TOK + 1 - q));
         const float2 acc = __fadd2_rn(acc0, acc1);
         l += acc.x + acc.y;
@@ -331,7 +374,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
   } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegOther) : "memory");
     if (!skip && warp == 8) {
       // ------------------------------------------------------------------------ TMA producer
       const int R = p.box_rows, nb = BN / R;             // page boxes per K/V tile (<= BN/16)
@@ -352,15 +395,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         m0 + qt * kBM, bar(L::B_Q));
       }
       // Physical row of box b of tile t (past the pool -- TMA fills zeros -- beyond n_max).
+      int* const pt_s = reinterpret_cast<int*>(base_ptr + L::PT_OFF);
+      const int n_cached = cache_page_table(p, pt_s, n_max, lane);
       auto box_row = [&](int t, int b) -> int {
         const int tok = t * BN + b * R;
         if (b >= nb || t >= nk || tok >= n_max) return p.total_rows;
-        int pg = __ldg(p.page_table + tok / p.page_size);
-        if (pg < 0 || pg >= p.num_pages) {
-          atomicCAS(p.status, 0, 5 /* WF_ERR_PAGE_OOB */);
-          pg = 0;
-        }
-        return pg * p.page_size + tok % p.page_size;
+        return pool_row(p, pt_s, n_cached, tok);
       };
       // Tiles are also prefetched into L2 kPrefetchKeys ahead: every CTA of a head streams the
       // same K/V at about the same time, so without it each tile would wait on an HBM round trip.
@@ -478,7 +518,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int q = 0; q < kNQT; ++q) {
           if (!mbar_wait(bar(L::B_P + NSB * q + j % NSB), (j / NSB) & 1, w)) return false;
           tc_fence_after();
-          const uint32_t pa = tmem + static_cast<uint32_t>(q * 128 + BN * (j % NSB));
+          const uint32_t pa = tmem + kPCol + static_cast<uint32_t>(q * 128 + BN * (j % NSB));
           const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
   #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)      // 16 keys = 8 TMEM columns / 2 KB of V
@@ -490,6 +530,74 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         return true;
       };
 
+#if WF_MMA_ORDER == 1
+      static_assert(WF_MMA_ORDER != 1 || BN == 128, "the staggered order assumes 128-key tiles");
+      // Staggered order: ... P.V_0(j), S_0(j+1), P.V_1(j), S_1(j+1) ...  The softmax of one Q
+      // tile then runs while the tensor pipe works on the other tile.  S_q(j+1) is issued as two
+      // 64-key halves: the first writes TMEM columns 0..63, which P.V_q(j) does not read (P
+      // sits in columns 64..127), so it goes straight after P.V_q(j); only the second half
+      // waits for P.V_q(j) to complete, and the first half keeps the pipe busy meanwhile.
+      constexpr uint32_t idesc_qh = idesc_bf16_f32(kBM, 64, 0, 0);
+      auto issue_s_half = [&](int j, int q, int half) {
+        const int slot = (2 * j) % NS;
+        const uint64_t dk = dk0 + ((static_cast<uint32_t>(slot) * KTILE + half * 64u * 128u) >> 4);
+        const uint32_t sd = tmem + static_cast<uint32_t>(q * 128 + 64 * half);
+        const uint64_t dq = dq0 + ((static_cast<uint32_t>(q) * QTILE) >> 4);
+  #pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(sd, dq + (((kk / 4) * QHALF + (kk % 4) * 32) >> 4),
+                  dk + (((kk / 4) * KHALF + (kk % 4) * 32) >> 4), idesc_qh, kk > 0 ? 1u : 0u);
+      };
+      auto wait_k = [&](int j) -> bool {
+        const int it = 2 * j;
+        if (!mbar_wait(bar(L::B_KVF + it % NS), (it / NS) & 1, w)) return false;
+        tc_fence_after();
+        return true;
+      };
+      if (ok) ok = wait_k(0);
+      if (ok) {
+  #pragma unroll 1
+        for (int q = 0; q < kNQT; ++q) {
+          issue_s_half(0, q, 0);
+          issue_s_half(0, q, 1);
+          umma_commit(bar(L::B_S + q));
+        }
+        umma_commit(bar(L::B_KVE + 0));
+      }
+      for (int j = 0; ok && j < nk; ++j) {
+        const int itv = 2 * j + 1, slotv = itv % NS;
+        ok = mbar_wait(bar(L::B_KVF + slotv), (itv / NS) & 1, w);
+        if (ok && j == nk - 1 && zero_tail) ok = mbar_wait(bar(L::B_VZ), 0, w);
+        const uint64_t dv = dv0 + ((static_cast<uint32_t>(slotv) * KTILE) >> 4);
+  #pragma unroll 1
+        for (int q = 0; q < kNQT && ok; ++q) {
+          ok = mbar_wait(bar(L::B_P + q), j & 1, w);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t pa = tmem + kPCol + static_cast<uint32_t>(q * 128);
+          const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
+  #pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_ts(od, pa + 8u * kk, dv + ((kk * 2048u) >> 4), idesc_pv,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar(L::B_O + q));
+          if (q == kNQT - 1) umma_commit(bar(L::B_KVE + slotv));   // V_j free
+          if (j + 1 < nk) {
+            if (q == 0) ok = wait_k(j + 1);
+            if (!ok) break;
+            issue_s_half(j + 1, q, 0);
+            ok = mbar_wait(bar(L::B_O + q), j & 1, w);              // P.V_q(j) done reading P
+            if (!ok) break;
+            tc_fence_after();
+            issue_s_half(j + 1, q, 1);
+            umma_commit(bar(L::B_S + q));
+            if (q == kNQT - 1) umma_commit(bar(L::B_KVE + (2 * (j + 1)) % NS));   // K_{j+1} free
+          }
+        }
+      }
+      (void)issue_s;
+      (void)issue_pv;
+#else
       // With two S buffers, QK^T of tile j+1 is issued before P.V of tile j so the tensor pipe
       // has work while the softmax of tile j runs.
       if (ok) ok = issue_s(0);
@@ -498,6 +606,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (ok) ok = issue_pv(j);
         if (NSB == 1 && ok && j + 1 < nk) ok = issue_s(j + 1);
       }
+#endif
       // every MMA this thread issued must complete before TMEM is released
       umma_commit(bar(L::B_DRAIN));
       mbar_wait_drain(bar(L::B_DRAIN), 0);

@@ -13,6 +13,7 @@
 #include "../../include/wf.h"
 #include "append_kernel.cuh"
 #include "attn_kernel.cuh"
+#include "attn_pair_kernel.cuh"
 
 // First error any kernel of this library recorded on this device (0 = none); cleared by
 // wf_check_status.
@@ -20,6 +21,10 @@ __device__ int g_wf_status = 0;
 // Launch id of the last attention launch in which a bounded wait ran out; every other CTA of
 // that launch stops as soon as it sees it.
 __device__ unsigned g_wf_abort = 0;
+
+#ifndef WF_ATTN_PAIR
+#define WF_ATTN_PAIR 0
+#endif
 
 namespace {
 
@@ -64,7 +69,10 @@ int device_state(DeviceState** out) {
                                  wfk::AttnSmem<128, wfk::kBN>::ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<64, wfk::kBN>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 wfk::AttnSmem<64, wfk::kBN>::ALLOC) != cudaSuccess) {
+                                 wfk::AttnSmem<64, wfk::kBN>::ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(wfk::wf_attn_pair_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 wfk::PairSmem::ALLOC) != cudaSuccess) {
           cudaGetLastError();
           return WF_ERR_CUDA;
         }
@@ -155,6 +163,23 @@ int gcd_int(int a, int b) {
   return a;
 }
 
+// One CTA waits on a barrier nobody arrives on; the bounded wait must give up, record
+// WF_ERR_TIMEOUT and return.
+__global__ void wf_selftest_timeout_kernel(int* status, unsigned* grid_abort, unsigned launch_id,
+                                           unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t never;
+  __shared__ int cta_abort;
+  if (threadIdx.x == 0) {
+    cta_abort = 0;
+    wfk::mbar_init(wfk::smem_u32(&never), 1);
+    wfk::mbar_init_fence();
+  }
+  __syncthreads();
+  const wfk::WaitCtx w{&cta_abort, grid_abort, status, launch_id, WF_ERR_TIMEOUT, timeout_ns};
+  if (threadIdx.x == 0) (void)wfk::mbar_wait(wfk::smem_u32(&never), 0, w);
+  __syncthreads();
+}
+
 }  // namespace
 
 extern "C" {
@@ -228,14 +253,18 @@ int wf_attn_forward(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* 
   static_assert(alignof(wfk::AttnParams) >= 64, "tensor maps need 64-byte alignment");
   wfk::AttnParams p;
   std::memset(&p, 0, sizeof(p));
-  const int box_rows = gcd_int(ps, wfk::kBN);   // a box never crosses a page or a tile edge
+  // CTA pairs run head_dim 128; a box never crosses a page or a tile edge
+  const bool use_pair = (D == 128) && WF_ATTN_PAIR;
+  const int box_rows = gcd_int(ps, use_pair ? 64 : wfk::kBN);
+  const int box_rows_v = gcd_int(ps, use_pair ? wfk::kPairBN : wfk::kBN);
   const int64_t total_rows = static_cast<int64_t>(kv_pages->num_pages) * ps;
   if (!encode_rows(&p.tm_q, q, D, H, t_q, wfk::kBM, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
       !encode_rows(&p.tm_k, kv_pages->k_pool, D, H, total_rows, box_rows,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
-      !encode_rows(&p.tm_v, kv_pages->v_pool, D, H, total_rows, box_rows,
+      !encode_rows(&p.tm_v, kv_pages->v_pool, D, H, total_rows, box_rows_v,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
     return WF_ERR_CUDA;
+  p.box_rows_v = box_rows_v;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse_or_null;
   p.page_table = page_table_row;
@@ -261,14 +290,29 @@ int wf_attn_forward(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* 
   p.nqc = nqc;
 
   const int64_t grid = static_cast<int64_t>(p.n_pairs) * H;
-  if (grid > INT32_MAX) return WF_ERR_SHAPE;
+  if (2 * grid > INT32_MAX) return WF_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (D == 128)
+  if (use_pair)
+    wfk::wf_attn_pair_kernel<<<static_cast<unsigned>(2 * grid), wfk::kPairThreads,
+                               wfk::PairSmem::ALLOC, s>>>(p);
+  else if (D == 128)
     wfk::wf_attn_fwd_kernel<128, wfk::kBN><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
                                              wfk::AttnSmem<128, wfk::kBN>::ALLOC, s>>>(p);
   else
     wfk::wf_attn_fwd_kernel<64, wfk::kBN><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
                                             wfk::AttnSmem<64, wfk::kBN>::ALLOC, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_selftest_timeout(unsigned timeout_us, wf_stream_t stream) {
+  if (timeout_us < 1 || timeout_us > 1000000) return WF_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  const int rc = device_state(&d);
+  if (rc) return rc;
+  unsigned id = g_launch_counter.fetch_add(1);
+  if (id == 0) id = g_launch_counter.fetch_add(1);
+  wf_selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      d->status, d->abort_word, id, 1000ull * timeout_us);
   return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 

@@ -137,6 +137,16 @@ int wf_attn_forward(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* 
  */
 int wf_check_status(wf_stream_t stream);
 
+/*
+ * wf_selftest_timeout -- exercise the kernels' failure path without faulting anything: one CTA
+ * waits, through the same bounded mbarrier wait the attention kernels use, on a barrier that no
+ * thread will ever arrive on.  After `timeout_us` microseconds (1..1000000) the wait gives up,
+ * records WF_ERR_TIMEOUT in the device status word and the kernel returns normally; the CUDA
+ * context stays usable.  Asynchronous on `stream`; read the result with wf_check_status.
+ * (No counterpart on the reference pages: it exists so the timeout path can be tested.)
+ */
+int wf_selftest_timeout(unsigned timeout_us, wf_stream_t stream);
+
 /* wf_strerror -- a static, human-readable name for an error code. */
 const char* wf_strerror(int code);
 

@@ -105,6 +105,11 @@ def test_validation_errors_without_a_gpu(abi):
     assert _append(abi, _pool(abi), ok_desc, k=FAKE + 4) == abi.WF_ERR_INVALID_ARG
 
 
+def test_selftest_timeout_rejects_bad_limits(abi):
+    assert abi.lib.wf_selftest_timeout(0, None) == abi.WF_ERR_INVALID_ARG
+    assert abi.lib.wf_selftest_timeout(2000000, None) == abi.WF_ERR_INVALID_ARG
+
+
 def test_empty_work_is_a_no_op(abi):
     """T_q = 0 and empty chunks return WF_OK before any device work."""
     desc = abi.WavefrontDesc([0, 64, 64], [0, 0], 1, 8)        # the only query chunk is empty

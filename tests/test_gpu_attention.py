@@ -186,3 +186,21 @@ def test_out_of_range_page_in_attention_is_reported():
     run(layer, q)
     assert check_status() == WF_ERR_PAGE_OOB
     assert check_status() == WF_OK
+
+
+def test_bounded_wait_runs_out_and_context_survives():
+    """A kernel wait that nothing completes gives up after its limit, reports WF_ERR_TIMEOUT,
+    and the device keeps working: the next attention call is still correct."""
+    from block_causal_streaming_b200 import WF_ERR_TIMEOUT, selftest_timeout
+    import time
+    t0 = time.perf_counter()
+    selftest_timeout(20000)                     # 20 ms
+    assert check_status() == WF_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    assert check_status() == WF_OK
+    wl = CONFIGS[1]
+    inp = make_inputs(wl)
+    layer, q, _, _ = place(wl, inp)
+    out = run(layer, q)
+    assert check_status() == WF_OK
+    assert_parity(out.float().cpu().numpy(), full_oracle(wl, inp, with_lse=False), "after timeout")
