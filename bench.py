@@ -39,8 +39,10 @@ from block_causal_streaming_b200.workloads import CONFIGS, Workload, make_inputs
 
 METRIC = "block-causal chunk-attention TFLOP/s and % of B200 bf16 peak; tokens/s"
 UNIT = "TFLOP/s"
+# the attention kernel and the host code that sets up its launch (tensor-map boxes, grid order)
 KERNEL_SOURCES = ["block_causal_streaming_b200/csrc/attn_kernel.cuh",
-                  "block_causal_streaming_b200/csrc/sm100.cuh"]
+                  "block_causal_streaming_b200/csrc/sm100.cuh",
+                  "block_causal_streaming_b200/csrc/wf_api.cu"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

@@ -10,36 +10,36 @@
 // One CTA = one unit of work: a head and 256 consecutive query rows (two 128-row Q tiles that
 // share every K/V tile they load).  Units are numbered so that the hardware's in-order block
 // dispatch runs the most expensive first (longest-processing-time order): kv_end is
-// non-decreasing in the query row, so the last query rows have the most visible keys; blockIdx 0
-// takes the last 256 rows, heads vary fastest.
+// non-decreasing in the query row, so blockIdx 0 takes the last 256 rows.  Heads vary fastest, so
+// the CTAs of all heads stream the same key range at about the same time and share it in L2.
 //
 // Warp roles (384 threads):
 //   warps 0-3  softmax of Q tile 0: thread t owns query row t (TMEM lane t)
 //   warps 4-7  softmax of Q tile 1
-//   warp  8    TMA producer: Q tiles once, then K_j, V_j (BN keys each) into a ring of NS
+//   warp  8    TMA producer: Q tiles once, then K_j, V_j (128 keys each) into a ring of NS
 //              shared-memory slots, page by page through the page table; zeroes the rows of
 //              the last V tile past the last visible key; allocates/frees TMEM
 //   warp  9    MMA issuer (one thread): S_q = Q_q K_j^T (SS form) and O_q += P_q V_j (TS form,
-//              P in TMEM), in a fixed order; with two S buffers QK^T of tile j+1 goes before
-//              P.V of tile j
+//              P in TMEM)
 //   warps 10-11 idle
-// TMEM (512 columns): per Q tile q, NSB = 128/BN S buffers of BN fp32 columns, S_q[b] at
-// 128q + BN b (P_q of a tile, bf16x2, overwrites the first BN/2 columns of its own S buffer), and
-// O_q at 256 + Dq.  With BN = 64 the two S buffers let the softmax of tile j run while QK^T of
-// tile j+1 is computed; with BN = 128 there is one buffer and the chain is serial.
+// TMEM (512 columns): S_q at 128 q (128 fp32 columns; P_q, bf16x2, overwrites its first 64) and
+// O_q at 256 + D q.
+//
+// Issue order: S_0(0), S_1(0), then for every tile j: P.V_0(j), S_0(j+1), P.V_1(j), S_1(j+1).
+// The two Q tiles run half a period apart: while the softmax of one tile computes P, the tensor
+// pipe works on the other tile's P.V and QK^T, and the two softmax warpgroups do not compete for
+// the exp unit at the same time.  S_q(j+1) overwrites the columns P.V_q(j) reads P from; PTX
+// orders consecutive MMAs only for the same accumulator, so S_q(j+1) is issued after o_done[q]
+// reports that P.V_q(j) completed.
 //
 // Synchronisation (all mbarriers, all waits bounded):
 //   q_full          TMA -> MMA          Q tiles landed
 //   kv_full[s]      TMA -> MMA          K or V tile landed in slot s
 //   kv_empty[s]     MMA commit -> TMA   slot s free again (both Q tiles' MMAs on it completed)
-//   s_full[q][b]    MMA commit -> softmax q   S of tile j (b = j mod NSB) ready
-//   p_full[q][b]    softmax q -> MMA    P of tile j written to TMEM (and O_q rescaled if needed)
-//   o_done[q][b]    MMA commit -> MMA / softmax   P.V of tile j (b = j mod NSB) completed
+//   s_full[q]       MMA commit -> softmax q   S_q of the current tile ready
+//   p_full[q]       softmax q -> MMA    P_q written to TMEM (and O_q rescaled if needed)
+//   o_done[q]       MMA commit -> MMA / softmax   P.V_q of the current tile completed
 //   v_zeroed        TMA warp -> MMA     tail rows of the last V tile zeroed
-// S of tile j+NSB overwrites the columns P.V of tile j reads P from; the PTX ordering guarantee
-// between consecutive MMAs covers only the same accumulator, so the MMA warp issues it only after
-// o_done[q][b] reports that P.V completed.  The softmax rescales O only after P.V of the
-// previous tile completed.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -49,27 +49,14 @@
 namespace wfk {
 
 constexpr int kBM = 128;        // query rows per Q tile (UMMA M)
-#ifndef WF_ATTN_BN
-#define WF_ATTN_BN 128
-#endif
 #ifndef WF_EXP2_POLY_EIGHTHS
-#define WF_EXP2_POLY_EIGHTHS 2   // column pairs out of 8 whose exp2 runs on the FMA pipe
-#endif
-#ifndef WF_MMA_ORDER
-#define WF_MMA_ORDER 0   // 1: staggered Q tiles, QK^T issued as two 64-key halves, P in columns 64..127
-#endif
-#ifndef WF_SOFTMAX_PINGPONG
-#define WF_SOFTMAX_PINGPONG 0     // 1: the two softmax warpgroups take turns on the exp phase
-#endif
-#ifndef WF_UNIT_ORDER
-#define WF_UNIT_ORDER 0
+#define WF_EXP2_POLY_EIGHTHS 0   // column pairs out of 8 whose exp2 runs on the FMA pipe
 #endif
 #ifndef WF_KV_RING_KB
-#define WF_KV_RING_KB 128
+#define WF_KV_RING_KB 160   // K/V ring: 5 tiles of 32 KB at head_dim 128
 #endif
-constexpr int kBN = WF_ATTN_BN;  // keys per K/V tile (UMMA N of QK^T, K of PV): 64 or 128
+constexpr int kBN = 128;        // keys per K/V tile (UMMA N of QK^T, K of P.V)
 constexpr int kNQT = 2;         // Q tiles per CTA
-constexpr uint32_t kPCol = WF_MMA_ORDER == 1 ? 64u : 0u;   // TMEM column of P within its S buffer
 constexpr int kAttnThreads = 384;
 #ifndef WF_REG_SOFTMAX
 #define WF_REG_SOFTMAX 208
@@ -86,10 +73,6 @@ constexpr int kMaxQChunks = 64;
 #define WF_PT_CACHE 0      // 0: each tile reads its page-table entries from global memory
 #endif
 constexpr int kPtCache = WF_PT_CACHE;   // page-table entries a producer keeps in shared memory
-#ifndef WF_PREFETCH_KEYS
-#define WF_PREFETCH_KEYS 0
-#endif
-constexpr int kPrefetchKeys = WF_PREFETCH_KEYS;  // L2 prefetch distance of the K/V stream (0: off)
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;   // 0.2 s when draining
 
@@ -151,9 +134,9 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-template <int D, int BN>
+template <int D>
 struct AttnSmem {
-  static constexpr int NSB = 128 / BN;                   // S buffers per Q tile
+  static constexpr int BN = kBN;
   static constexpr int DH = D / 64;                      // 128-byte halves of a row
   static constexpr int NS = WF_KV_RING_KB * 1024 / (int)(DH * BN * 128);   // K/V ring slots
   static constexpr uint32_t QHALF = kBM * 128u;          // 128 rows x 128 B, 128B-swizzled
@@ -163,21 +146,22 @@ struct AttnSmem {
   static constexpr uint32_t Q_OFF = 0;
   static constexpr uint32_t KV_OFF = Q_OFF + kNQT * QTILE;
   static constexpr uint32_t BAR_OFF = KV_OFF + NS * KTILE;
-  // barrier indices; per-(q, b) barriers at base + NSB q + b
+  // barrier indices; per-Q-tile barriers at base + q
   static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NS, B_S = 1 + 2 * NS,
-                       B_P = B_S + 2 * NSB, B_O = B_P + 2 * NSB, B_DRAIN = B_O + 2 * NSB,
-                       B_VZ = B_DRAIN + 1, B_TOK = B_VZ + 1, NBAR = B_TOK + 2;
+                       B_P = B_S + kNQT, B_O = B_P + kNQT, B_DRAIN = B_O + kNQT,
+                       B_VZ = B_DRAIN + 1, NBAR = B_VZ + 1;
   static constexpr uint32_t PT_OFF = BAR_OFF + NBAR * 8;   // page-table cache
   static constexpr uint32_t MISC_OFF = PT_OFF + kPtCache * 4;
   static constexpr uint32_t BYTES = MISC_OFF + 16;
   static constexpr uint32_t ALLOC = BYTES + 1024;        // slack for 1024-byte alignment
+  static_assert(ALLOC <= 227u * 1024u, "shared memory per CTA exceeds 227 KB");
 };
 
-template <int D, int BN>
+template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     wf_attn_fwd_kernel(const __grid_constant__ AttnParams p) {
-  using L = AttnSmem<D, BN>;
-  constexpr int DH = L::DH, NS = L::NS, NSB = L::NSB;
+  using L = AttnSmem<D>;
+  constexpr int BN = L::BN, DH = L::DH, NS = L::NS;
   constexpr uint32_t QTILE = L::QTILE, QHALF = L::QHALF, KTILE = L::KTILE, KHALF = L::KHALF;
 
   extern __shared__ uint8_t smem_raw[];
@@ -190,13 +174,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int unit = blockIdx.x;
-#if WF_UNIT_ORDER == 1
-  const int pair = p.n_pairs - 1 - unit % p.n_pairs;    // head-major: one head's K/V live at once
-  const int head = unit / p.n_pairs;
-#else
   const int pair = p.n_pairs - 1 - unit / p.H;
   const int head = unit % p.H;
-#endif
   const int m0 = pair * (kNQT * kBM);
   const int last_row = min(m0 + kNQT * kBM, p.T_q) - 1;
   const int n_max = kv_end_of_row(p, last_row);        // keys any row of this unit may see
@@ -208,7 +187,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     *cta_abort = (*reinterpret_cast<volatile unsigned*>(p.grid_abort) == p.launch_id) ? 1 : 0;
     for (int i = 0; i < L::NBAR; ++i)
-      mbar_init(bar(i), ((i >= L::B_P && i < L::B_O) || i >= L::B_TOK) ? 128u : 1u);
+      mbar_init(bar(i), (i >= L::B_P && i < L::B_O) ? 128u : 1u);
     mbar_init_fence();
   }
   if (warp == 8) {
@@ -231,18 +210,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int row_g = m0 + q * kBM + row;                 // query row
       const int n_r = kv_end_of_row(p, min(row_g, p.T_q - 1));
       const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-      const uint32_t tS0 = tmem + lane_off + static_cast<uint32_t>(q * 128);
+      const uint32_t tS = tmem + lane_off + static_cast<uint32_t>(q * 128);
       const uint32_t tO = tmem + lane_off + 256u + static_cast<uint32_t>(q * D);
       const float sl2 = p.sl2;
       float m2 = -INFINITY;   // running max of the base-2 logits in use
       float l = 0.f;          // running sum of exp2(t - m2)
       bool ok = true;
       const float2 sl2x2 = make_float2(sl2, sl2);
-      if (WF_SOFTMAX_PINGPONG && q == 1) mbar_arrive(bar(L::B_TOK + 0));   // warpgroup 0 goes first
       for (int j = 0; j < nk; ++j) {
-        const int b = j % NSB;
-        const uint32_t tS = tS0 + static_cast<uint32_t>(BN * b);
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_S + NSB * q + b), (j / NSB) & 1, w));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_S + q), j & 1, w));
         if (!ok) break;
         tc_fence_after();
         float s[BN];
@@ -282,9 +258,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // O_q holds P.V of tiles < j once P.V of tile j-1 has completed; rescale this warp's
           // rows (threads whose max did not move multiply by 1).
-          const int bp = (j - 1) % NSB;
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(bar(L::B_O + NSB * q + bp), ((j - 1) / NSB) & 1, w));
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_O + q), (j - 1) & 1, w));
           if (!ok) break;
           tc_fence_after();
   #pragma unroll
@@ -298,15 +272,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         l *= alpha;
-        // p = exp2(s * scale * log2 e - m2) two columns at a time.  On unmasked tiles 3 of every
-        // 8 column pairs use the FMA-pipe polynomial and the rest the MUFU unit, which alone
-        // would be as slow as the tensor core at head_dim 128.  Masked tiles use the MUFU unit
-        // only, so masked columns give exactly 0.
-        if (WF_SOFTMAX_PINGPONG) {
-          // take turns with the other Q tile's warpgroup on the exp phase (token j of this one)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_TOK + q), j & 1, w));
-          if (!ok) break;
-        }
+        // p = exp2(s * scale * log2 e - m2) two columns at a time.  On unmasked tiles
+        // WF_EXP2_POLY_EIGHTHS of every 8 column pairs use the FMA-pipe polynomial and the rest
+        // the MUFU unit.  Masked tiles use the MUFU unit only, so masked columns give exactly 0.
         const float2 negm = make_float2(-m2, -m2);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         uint32_t pk[BN / 2];
@@ -335,18 +303,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
   #pragma unroll
         for (int h = 0; h < BN / 64; ++h)
-          tmem_st32(tS + kPCol + 32u * h, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h]));
-        if (WF_SOFTMAX_PINGPONG) mbar_arrive(bar(L::B_TOK + 1 - q));
+          tmem_st32(tS + 32u * h, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h]));
         const float2 acc = __fadd2_rn(acc0, acc1);
         l += acc.x + acc.y;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(L::B_P + NSB * q + b));
+        mbar_arrive(bar(L::B_P + q));
       }
       // ------------------------------------------------------------------------- epilogue
       if (ok)
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(bar(L::B_O + NSB * q + (nk - 1) % NSB), ((nk - 1) / NSB) & 1, w));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_O + q), (nk - 1) & 1, w));
       if (ok) {
         tc_fence_after();
         const float inv_l = 1.f / l;
@@ -402,23 +368,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (b >= nb || t >= nk || tok >= n_max) return p.total_rows;
         return pool_row(p, pt_s, n_cached, tok);
       };
-      // Tiles are also prefetched into L2 kPrefetchKeys ahead: every CTA of a head streams the
-      // same K/V at about the same time, so without it each tile would wait on an HBM round trip.
-      constexpr int PF = kPrefetchKeys / BN;
-      auto prefetch_tile = [&](int t, int row) {            // row: this lane's box row of tile t
-        if (PF > 0 && lane < nb && row < p.total_rows) {
-  #pragma unroll
-          for (int h = 0; h < DH; ++h) {
-            tma_prefetch_l2_3d(&p.tm_k, 64 * h, head, row);
-            tma_prefetch_l2_3d(&p.tm_v, 64 * h, head, row);
-          }
-        }
-      };
-      for (int t = 1; t < PF && t < nk; ++t) prefetch_tile(t, box_row(t, lane));
-      (void)prefetch_tile;
       for (int j = 0; j < nk && ok; ++j) {
         const int coord = box_row(j, lane);                 // lane b resolves box b of tile j
-        if (PF > 0) prefetch_tile(j + PF, box_row(j + PF, lane));
         int cb[BN / 16];
   #pragma unroll
         for (int b = 0; b < BN / 16; ++b) cb[b] = __shfl_sync(0xffffffffu, coord, b);
@@ -486,67 +437,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool zero_tail = (n_max - (nk - 1) * BN) < BN;   // the loader zeroes V's tail rows
       bool ok = mbar_wait(bar(L::B_Q), 0, w);
 
-      // S_q(j) = Q_q K_j^T into S buffer j mod NSB, once P.V of tile j-NSB has released it.
-      auto issue_s = [&](int j) -> bool {
-        const int it = 2 * j, slot = it % NS;
-        if (!mbar_wait(bar(L::B_KVF + slot), (it / NS) & 1, w)) return false;
-        const uint64_t dk = dk0 + ((static_cast<uint32_t>(slot) * KTILE) >> 4);
-  #pragma unroll
-        for (int q = 0; q < kNQT; ++q) {
-          if (j >= NSB &&
-              !mbar_wait(bar(L::B_O + NSB * q + j % NSB), ((j - NSB) / NSB) & 1, w))
-            return false;
-          tc_fence_after();
-          const uint32_t sd = tmem + static_cast<uint32_t>(q * 128 + BN * (j % NSB));
-          const uint64_t dq = dq0 + ((static_cast<uint32_t>(q) * QTILE) >> 4);
-  #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)   // 16 bf16 = 32 B per K-step; 64 per 128-B half
-            umma_ss(sd, dq + (((kk / 4) * QHALF + (kk % 4) * 32) >> 4),
-                    dk + (((kk / 4) * KHALF + (kk % 4) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
-          umma_commit(bar(L::B_S + NSB * q + j % NSB));
-        }
-        umma_commit(bar(L::B_KVE + slot));          // K_j free once both Q tiles' MMAs finish
-        return true;
-      };
-      // O_q += P_q(j) V_j, P read from TMEM (the first BN/2 columns of S buffer j mod NSB).
-      auto issue_pv = [&](int j) -> bool {
-        const int it = 2 * j + 1, slot = it % NS;
-        if (!mbar_wait(bar(L::B_KVF + slot), (it / NS) & 1, w)) return false;
-        if (j == nk - 1 && zero_tail && !mbar_wait(bar(L::B_VZ), 0, w)) return false;
-        const uint64_t dv = dv0 + ((static_cast<uint32_t>(slot) * KTILE) >> 4);
-  #pragma unroll
-        for (int q = 0; q < kNQT; ++q) {
-          if (!mbar_wait(bar(L::B_P + NSB * q + j % NSB), (j / NSB) & 1, w)) return false;
-          tc_fence_after();
-          const uint32_t pa = tmem + kPCol + static_cast<uint32_t>(q * 128 + BN * (j % NSB));
-          const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
-  #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)      // 16 keys = 8 TMEM columns / 2 KB of V
-            umma_ts(od, pa + 8u * kk, dv + ((kk * 2048u) >> 4), idesc_pv,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(bar(L::B_O + NSB * q + j % NSB));
-        }
-        umma_commit(bar(L::B_KVE + slot));          // V_j free once both P.V finish
-        return true;
-      };
-
-#if WF_MMA_ORDER == 1
-      static_assert(WF_MMA_ORDER != 1 || BN == 128, "the staggered order assumes 128-key tiles");
-      // Staggered order: ... P.V_0(j), S_0(j+1), P.V_1(j), S_1(j+1) ...  The softmax of one Q
-      // tile then runs while the tensor pipe works on the other tile.  S_q(j+1) is issued as two
-      // 64-key halves: the first writes TMEM columns 0..63, which P.V_q(j) does not read (P
-      // sits in columns 64..127), so it goes straight after P.V_q(j); only the second half
-      // waits for P.V_q(j) to complete, and the first half keeps the pipe busy meanwhile.
-      constexpr uint32_t idesc_qh = idesc_bf16_f32(kBM, 64, 0, 0);
-      auto issue_s_half = [&](int j, int q, int half) {
+      // S_q(j) = Q_q K_j^T: D/16 K-steps of 16 columns (4 per 128-byte half of a row).
+      auto issue_s_q = [&](int j, int q) {
         const int slot = (2 * j) % NS;
-        const uint64_t dk = dk0 + ((static_cast<uint32_t>(slot) * KTILE + half * 64u * 128u) >> 4);
-        const uint32_t sd = tmem + static_cast<uint32_t>(q * 128 + 64 * half);
+        const uint64_t dk = dk0 + ((static_cast<uint32_t>(slot) * KTILE) >> 4);
+        const uint32_t sd = tmem + static_cast<uint32_t>(q * 128);
         const uint64_t dq = dq0 + ((static_cast<uint32_t>(q) * QTILE) >> 4);
   #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           umma_ss(sd, dq + (((kk / 4) * QHALF + (kk % 4) * 32) >> 4),
-                  dk + (((kk / 4) * KHALF + (kk % 4) * 32) >> 4), idesc_qh, kk > 0 ? 1u : 0u);
+                  dk + (((kk / 4) * KHALF + (kk % 4) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+        umma_commit(bar(L::B_S + q));
       };
       auto wait_k = [&](int j) -> bool {
         const int it = 2 * j;
@@ -556,12 +457,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       };
       if (ok) ok = wait_k(0);
       if (ok) {
-  #pragma unroll 1
-        for (int q = 0; q < kNQT; ++q) {
-          issue_s_half(0, q, 0);
-          issue_s_half(0, q, 1);
-          umma_commit(bar(L::B_S + q));
-        }
+        issue_s_q(0, 0);
+        issue_s_q(0, 1);
         umma_commit(bar(L::B_KVE + 0));
       }
       for (int j = 0; ok && j < nk; ++j) {
@@ -574,7 +471,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           ok = mbar_wait(bar(L::B_P + q), j & 1, w);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t pa = tmem + kPCol + static_cast<uint32_t>(q * 128);
+          const uint32_t pa = tmem + static_cast<uint32_t>(q * 128);
           const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
   #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
@@ -584,29 +481,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (q == kNQT - 1) umma_commit(bar(L::B_KVE + slotv));   // V_j free
           if (j + 1 < nk) {
             if (q == 0) ok = wait_k(j + 1);
-            if (!ok) break;
-            issue_s_half(j + 1, q, 0);
-            ok = mbar_wait(bar(L::B_O + q), j & 1, w);              // P.V_q(j) done reading P
+            if (ok) ok = mbar_wait(bar(L::B_O + q), j & 1, w);      // P.V_q(j) done reading P
             if (!ok) break;
             tc_fence_after();
-            issue_s_half(j + 1, q, 1);
-            umma_commit(bar(L::B_S + q));
+            issue_s_q(j + 1, q);
             if (q == kNQT - 1) umma_commit(bar(L::B_KVE + (2 * (j + 1)) % NS));   // K_{j+1} free
           }
         }
       }
-      (void)issue_s;
-      (void)issue_pv;
-#else
-      // With two S buffers, QK^T of tile j+1 is issued before P.V of tile j so the tensor pipe
-      // has work while the softmax of tile j runs.
-      if (ok) ok = issue_s(0);
-      for (int j = 0; ok && j < nk; ++j) {
-        if (NSB > 1 && j + 1 < nk) ok = issue_s(j + 1);
-        if (ok) ok = issue_pv(j);
-        if (NSB == 1 && ok && j + 1 < nk) ok = issue_s(j + 1);
-      }
-#endif
       // every MMA this thread issued must complete before TMEM is released
       umma_commit(bar(L::B_DRAIN));
       mbar_wait_drain(bar(L::B_DRAIN), 0);

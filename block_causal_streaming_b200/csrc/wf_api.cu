@@ -64,12 +64,12 @@ int device_state(DeviceState** out) {
         if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_wf_status) != cudaSuccess ||
             cudaGetSymbolAddress(reinterpret_cast<void**>(&d.abort_word), g_wf_abort) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<128, wfk::kBN>,
+            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 wfk::AttnSmem<128, wfk::kBN>::ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<64, wfk::kBN>,
+                                 wfk::AttnSmem<128>::ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<64>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 wfk::AttnSmem<64, wfk::kBN>::ALLOC) != cudaSuccess ||
+                                 wfk::AttnSmem<64>::ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(wfk::wf_attn_pair_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  wfk::PairSmem::ALLOC) != cudaSuccess) {
@@ -296,11 +296,11 @@ int wf_attn_forward(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* 
     wfk::wf_attn_pair_kernel<<<static_cast<unsigned>(2 * grid), wfk::kPairThreads,
                                wfk::PairSmem::ALLOC, s>>>(p);
   else if (D == 128)
-    wfk::wf_attn_fwd_kernel<128, wfk::kBN><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
-                                             wfk::AttnSmem<128, wfk::kBN>::ALLOC, s>>>(p);
+    wfk::wf_attn_fwd_kernel<128><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
+                                   wfk::AttnSmem<128>::ALLOC, s>>>(p);
   else
-    wfk::wf_attn_fwd_kernel<64, wfk::kBN><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
-                                            wfk::AttnSmem<64, wfk::kBN>::ALLOC, s>>>(p);
+    wfk::wf_attn_fwd_kernel<64><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
+                                  wfk::AttnSmem<64>::ALLOC, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
