@@ -13,6 +13,10 @@ Printed (rank 0, one JSON line): throughput in TFLOP/s of algorithmic attention 
 with tokens/s, the roofline of the attention kernel, an end-to-end figure through the C ABI with
 host buffers, the CPU oracle as a baseline, and the SM clocks seen during the timed region.
 
+--config 3 / 5 run the other full-size wavefronts; --config wp runs one Wave-Parallelism rank's
+call (one 4680-token chunk against a 37 440-key prefix) through wf_attn_forward_split with the
+library's choice of key splits, whose timed attention then includes the merge kernel.
+
 With --gpus N > 1 (launched by torch.distributed.run) every rank runs an independent replica of
 the same workload: the path has no exchange step, so there is no data-path collective; a barrier
 and a max-reduction of the device times are the only collectives.
@@ -35,7 +39,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from block_causal_streaming_b200.workloads import CONFIGS, Workload, make_inputs  # noqa: E402
+from block_causal_streaming_b200.workloads import (CONFIGS, WP_RANK0, Workload,  # noqa: E402
+                                                   make_inputs)
 
 METRIC = "block-causal chunk-attention TFLOP/s and % of B200 bf16 peak; tokens/s"
 UNIT = "TFLOP/s"
@@ -47,6 +52,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ------------------------------------------------------------------------------ accounting
+def workload_of(config: str) -> Workload:
+    return WP_RANK0 if config == "wp" else CONFIGS[int(config)]
+
+
 def attention_flops(wl: Workload) -> int:
     """4 * D * H * sum over query rows of the number of keys that row may see."""
     off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
@@ -81,14 +90,15 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def load_traffic():
-    """DRAM bytes per attention launch from a committed ncu capture, if it matches this kernel."""
+def load_traffic(workload: str):
+    """DRAM bytes per attention launch from a committed ncu capture, if it matches this kernel
+    and workload."""
     path = os.path.join(ROOT, "profiles", "attn_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
-    if rec.get("kernel_hash") != kernel_hash():
+    if rec.get("kernel_hash") != kernel_hash() or rec.get("workload") != workload:
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -238,7 +248,7 @@ def gpu_arm(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     init_dist(world, "nccl")
-    wl = CONFIGS[args.config]
+    wl = workload_of(args.config)
     inp = make_inputs(wl)
     H, D = wl.heads, wl.head_dim
     off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
@@ -255,13 +265,15 @@ def gpu_arm(args, world, rank, local):
     active = list(range(nctx, wl.num_chunks))
     layer.append_range(k, v, range(nctx))            # clean context: published once
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = len(active) + 1
+    splits = 0 if args.config == "wp" else None       # library-chosen key splits
+    split_used = splits is not None and wf.attn_workspace_size(layer.desc, H, D, 0) > 0
+    launches_per_step = len(active) + 1 + (1 if split_used else 0)
 
     def step(ev_pair=None):
         layer.append_range(k, v, active)
         if ev_pair is not None:
             ev_pair[0].record(stream)
-        layer.forward(q, out, scale=scale)
+        layer.forward(q, out, scale=scale, splits=splits)
         if ev_pair is not None:
             ev_pair[1].record(stream)
 
@@ -312,7 +324,7 @@ def gpu_arm(args, world, rank, local):
         for c in active:
             a, b = off[c] - base, off[c + 1] - base
             layer.append(c, k_act[a:b], v_act[a:b])
-        layer.forward(q_in, out, scale=scale)
+        layer.forward(q_in, out, scale=scale, splits=splits)
         out_h.copy_(out, non_blocking=True)
 
     for _ in range(max(1, min(args.warmup, 3))):
@@ -334,6 +346,8 @@ def gpu_arm(args, world, rank, local):
         raise RuntimeError(f"device status after end-to-end run: {wf.strerror(rc)}")
 
     peaks, peak_src = load_peaks()
+    touched_mb = (2 * q.numel() + 4 * (off[-1] - off[nctx]) * H * D + 2 * off[-1] * H * D) \
+        * 2 / 1e6   # q, out, appended K/V (read + written), K/V pages read
     step_s = elapsed_max / args.steps
     value = aggregate(flop, world, step_s) / 1e12
     attn_avg_s = statistics.mean(attn_ms) / 1e3
@@ -346,14 +360,19 @@ def gpu_arm(args, world, rank, local):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)*0.5 bf16)",
         "config": {"workload": wl.name, "heads": H, "head_dim": D, "t_q": wl.t_q,
                    "t_kv": wl.t_kv, "chunks": f"{nctx} ctx + {len(active)} active x 4680",
-                   "page_size": wl.page_size, "step": "append 5 active chunks + attention",
-                   "l2": "inputs larger than L2 (~490 MB touched per step vs 126 MB L2)",
+                   "page_size": wl.page_size,
+                   "step": f"append {len(active)} active chunks + attention"
+                           + (" (key splits + merge)" if split_used else ""),
+                   "l2": f"inputs larger than L2 (~{touched_mb:.0f} MB touched per step vs "
+                         "126 MB L2)",
                    "parallelism": f"replicas x{world}"},
         "tokens_per_s": round(world * wl.t_q / step_s, 1),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
-        "roofline": {"bound": "tensor", "kernel": "wf_attn_fwd_kernel<128>",
+        "roofline": {"bound": "tensor",
+                     "kernel": "wf_attn_fwd_kernel<128>"
+                               + (" + wf_combine_kernel<128>" if split_used else ""),
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": load_traffic(),
+                     "frac": round(achieved / peak, 4), "traffic": load_traffic(wl.name),
                      "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "attn_ms_avg": round(attn_avg_s * 1e3, 4),
                      "attn_ms_p50": round(statistics.median(attn_ms), 4)},
@@ -380,7 +399,7 @@ def reference_arm(args, world, rank):
     """The oracle as it stands, on the host cores, on bounded samples of the same workload."""
     if rank != 0:
         return None
-    wl = CONFIGS[args.config]
+    wl = workload_of(args.config)
     inp = make_inputs(wl)
     per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
     for i in range(args.warmup):
@@ -416,7 +435,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["wf", "reference"], default="wf")
-    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 5])
+    ap.add_argument("--config", default="2", choices=["2", "3", "5", "wp"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -26,7 +26,7 @@ WF_MAX_CHUNKS = 64
 
 # Every symbol include/wf.h declares (checked by the CPU tests).
 EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror", "wf_version",
-            "wf_selftest_timeout")
+            "wf_selftest_timeout", "wf_attn_forward_split", "wf_attn_workspace_size")
 
 
 class WfError(RuntimeError):
@@ -69,6 +69,14 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wf_version.restype = i32
     lib.wf_selftest_timeout.argtypes = [ctypes.c_uint, vp]
     lib.wf_selftest_timeout.restype = i32
+    lib.wf_attn_forward_split.argtypes = [vp, ctypes.POINTER(KvPool),
+                                          ctypes.POINTER(ctypes.c_int32),
+                                          ctypes.POINTER(Wavefront), ctypes.c_float, vp,
+                                          ctypes.POINTER(ctypes.c_float), i32, vp,
+                                          ctypes.c_size_t, vp]
+    lib.wf_attn_forward_split.restype = i32
+    lib.wf_attn_workspace_size.argtypes = [ctypes.POINTER(Wavefront), i32, i32, i32]
+    lib.wf_attn_workspace_size.restype = ctypes.c_size_t
     return lib
 
 
@@ -153,6 +161,36 @@ def attn_forward(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: fl
         _stream_handle(stream))
     if rc != WF_OK:
         raise WfError(rc, "wf_attn_forward")
+
+
+def attn_workspace_size(wf: WavefrontDesc, num_heads: int, head_dim: int, splits: int = 0) -> int:
+    """wf_attn_workspace_size: bytes of workspace attn_forward_split needs (0: none)."""
+    return int(lib.wf_attn_workspace_size(ctypes.byref(wf.c), int(num_heads), int(head_dim),
+                                          int(splits)))
+
+
+def attn_forward_split(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: float, out,
+                       splits: int = 0, workspace=None, lse=None, stream=None) -> None:
+    """wf_attn_forward_split: attn_forward with every unit's keys split over ``splits`` CTAs
+    (0: the library chooses) and merged; ``workspace`` is a device uint8 tensor of at least
+    attn_workspace_size(...) bytes (None when that is 0)."""
+    for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
+                    (page_table_row, "page_table_row", "i32"), (out, "out", "bf16")):
+        _check_tensor(t, n, d)
+    if lse is not None:
+        _check_tensor(lse, "lse", "f32")
+    pool = _pool_struct(k_pool, v_pool)
+    rc = lib.wf_attn_forward_split(
+        q.data_ptr(), ctypes.byref(pool),
+        ctypes.cast(ctypes.c_void_p(page_table_row.data_ptr()), ctypes.POINTER(ctypes.c_int32)),
+        ctypes.byref(wf.c), float(scale), out.data_ptr(),
+        ctypes.cast(ctypes.c_void_p(lse.data_ptr()), ctypes.POINTER(ctypes.c_float))
+        if lse is not None else None,
+        int(splits), workspace.data_ptr() if workspace is not None else None,
+        workspace.numel() * workspace.element_size() if workspace is not None else 0,
+        _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_attn_forward_split")
 
 
 def selftest_timeout(timeout_us: int, stream=None) -> None:

@@ -92,6 +92,11 @@ struct AttnParams {
   int nqc;                          // non-empty query chunks
   int qc_row_end[kMaxQChunks];      // exclusive end row of query chunk i (query-row space)
   int qc_kv_end[kMaxQChunks];       // number of visible keys for rows of query chunk i
+  // Key splits: with n_splits > 1 every unit runs as n_splits CTAs over consecutive parts of its
+  // key tiles, and each writes its normalised partial output and log-sum-exp instead of `out`.
+  int n_splits;
+  float* part_o;                    // fp32 [n_splits][T_q][H][D]
+  float* part_lse;                  // fp32 [n_splits][H][T_q], natural log; -inf: no key seen
 };
 
 __device__ __forceinline__ int kv_end_of_row(const AttnParams& p, int r) {
@@ -173,13 +178,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto bar = [&](int i) -> uint32_t { return base + L::BAR_OFF + 8u * static_cast<uint32_t>(i); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int unit = blockIdx.x;
+  const int unit = blockIdx.x / p.n_splits;
+  const int split = blockIdx.x - unit * p.n_splits;
   const int pair = p.n_pairs - 1 - unit / p.H;
   const int head = unit % p.H;
   const int m0 = pair * (kNQT * kBM);
   const int last_row = min(m0 + kNQT * kBM, p.T_q) - 1;
   const int n_max = kv_end_of_row(p, last_row);        // keys any row of this unit may see
-  const int nk = (n_max + BN - 1) / BN;                // K/V tiles to visit
+  const int n_tiles = (n_max + BN - 1) / BN;           // key tiles of the unit
+  // This CTA's part of them: tiles [kb, kb + nk).  The host keeps n_splits <= n_tiles of every
+  // unit, so nk >= 1.  Tile j below is local; its keys start at (kb + j) * BN.
+  const int kb = static_cast<int>(static_cast<int64_t>(split) * n_tiles / p.n_splits);
+  const int nk = static_cast<int>(static_cast<int64_t>(split + 1) * n_tiles / p.n_splits) - kb;
 
   const WaitCtx w{cta_abort, p.grid_abort, p.status, p.launch_id, 6 /* WF_ERR_TIMEOUT */,
                   kWaitTimeoutNs};
@@ -231,7 +241,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   #pragma unroll
           for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
         }
-        const int lim = n_r - j * BN;                       // visible columns of this tile
+        const int lim = n_r - (kb + j) * BN;                // visible columns of this tile
         const bool masked = lim < BN;
         if (masked) {
   #pragma unroll
@@ -275,7 +285,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // p = exp2(s * scale * log2 e - m2) two columns at a time.  On unmasked tiles
         // WF_EXP2_POLY_EIGHTHS of every 8 column pairs use the FMA-pipe polynomial and the rest
         // the MUFU unit.  Masked tiles use the MUFU unit only, so masked columns give exactly 0.
-        const float2 negm = make_float2(-m2, -m2);
+        // no visible key yet (possible in a later key split): every p is exactly 0
+        const float mref = m2 == -INFINITY ? 0.f : m2;
+        const float2 negm = make_float2(-mref, -mref);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         uint32_t pk[BN / 2];
         if (!masked) {
@@ -313,7 +325,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // ------------------------------------------------------------------------- epilogue
       if (ok)
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_O + q), (nk - 1) & 1, w));
-      if (ok) {
+      if (ok && p.n_splits > 1) {
+        // partial result of this key split: O / l in fp32 and its log-sum-exp (-inf, O = 0 if
+        // no key of this split is visible to the row)
+        tc_fence_after();
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        const bool live = row_g < p.T_q;
+        float* const prow =
+            p.part_o + ((static_cast<size_t>(split) * p.T_q + row_g) * p.H + head) * D;
+  #pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + 32u * c, r);
+          tmem_wait_ld();
+          if (live) {
+            float4* dst = reinterpret_cast<float4*>(prow + 32 * c);
+  #pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv_l,
+                                   __uint_as_float(r[4 * i + 1]) * inv_l,
+                                   __uint_as_float(r[4 * i + 2]) * inv_l,
+                                   __uint_as_float(r[4 * i + 3]) * inv_l);
+          }
+        }
+        if (live)
+          p.part_lse[(static_cast<size_t>(split) * p.H + head) * p.T_q + row_g] =
+              l > 0.f ? (m2 + __log2f(l)) * 0.69314718056f : -INFINITY;
+      } else if (ok) {
         tc_fence_after();
         const float inv_l = 1.f / l;
         const bool live = row_g < p.T_q;
@@ -364,7 +402,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int* const pt_s = reinterpret_cast<int*>(base_ptr + L::PT_OFF);
       const int n_cached = cache_page_table(p, pt_s, n_max, lane);
       auto box_row = [&](int t, int b) -> int {
-        const int tok = t * BN + b * R;
+        const int tok = (kb + t) * BN + b * R;
         if (b >= nb || t >= nk || tok >= n_max) return p.total_rows;
         return pool_row(p, pt_s, n_cached, tok);
       };
@@ -396,7 +434,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
       }
-      const int zero_from = n_max - (nk - 1) * BN;         // rows >= this of the last V tile
+      const int zero_from = n_max - (kb + nk - 1) * BN;    // rows >= this of the last V tile
       if (ok && zero_from < BN) {
         // Rows past the last visible key may hold anything (even NaN, which 0 * NaN would spread
         // through P.V); once the last V tile has landed, zero them and release the MMA warp.
@@ -434,7 +472,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dq0 = smem_desc_sw128(base + L::Q_OFF, 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(base + L::KV_OFF, 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(base + L::KV_OFF, KHALF, 1024);
-      const bool zero_tail = (n_max - (nk - 1) * BN) < BN;   // the loader zeroes V's tail rows
+      const bool zero_tail = (n_max - (kb + nk - 1) * BN) < BN;   // the loader zeroes V's tail
       bool ok = mbar_wait(bar(L::B_Q), 0, w);
 
       // S_q(j) = Q_q K_j^T: D/16 K-steps of 16 columns (4 per 128-byte half of a row).

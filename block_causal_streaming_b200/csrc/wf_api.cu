@@ -8,12 +8,14 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/wf.h"
 #include "append_kernel.cuh"
 #include "attn_kernel.cuh"
 #include "attn_pair_kernel.cuh"
+#include "combine_kernel.cuh"
 
 // First error any kernel of this library recorded on this device (0 = none); cleared by
 // wf_check_status.
@@ -163,6 +165,195 @@ int gcd_int(int a, int b) {
   return a;
 }
 
+// ------------------------------------------------------------------------------ attention setup
+// The query chunks of a wavefront: rows of query chunk i end at row_end[i] (query-row space) and
+// see the first kv_end[i] keys.  Empty chunks own no rows and are skipped.
+struct QueryPlan {
+  int t_q = 0;
+  int nqc = 0;
+  int row_end[WF_MAX_CHUNKS];
+  int kv_end[WF_MAX_CHUNKS];
+};
+
+int query_plan(const wf_wavefront_t* wf, QueryPlan* qp) {
+  if (wf->chunk_offsets == nullptr || wf->num_chunks < 1 || wf->num_chunks > WF_MAX_CHUNKS ||
+      wf->num_ctx_chunks < 0 || wf->num_ctx_chunks >= wf->num_chunks)
+    return WF_ERR_SHAPE;
+  const int32_t* off = wf->chunk_offsets;
+  const int t_ctx = off[wf->num_ctx_chunks];
+  qp->nqc = 0;
+  for (int c = wf->num_ctx_chunks; c < wf->num_chunks; ++c) {
+    if (off[c + 1] < off[c]) return WF_ERR_SHAPE;
+    if (off[c + 1] == off[c]) continue;
+    qp->row_end[qp->nqc] = off[c + 1] - t_ctx;
+    qp->kv_end[qp->nqc] = off[c + 1];
+    ++qp->nqc;
+  }
+  qp->t_q = off[wf->num_chunks] - t_ctx;
+  return WF_OK;
+}
+
+constexpr int kUnitRows = wfk::kNQT * wfk::kBM;   // query rows per unit (one CTA)
+constexpr int kMaxSplits = 16;
+
+int num_pairs(const QueryPlan& qp) { return (qp.t_q + kUnitRows - 1) / kUnitRows; }
+
+// Key tiles of the units of row block `pair` (the block's last row sees the most keys).
+int unit_tiles(const QueryPlan& qp, int pair) {
+  const int last = std::min((pair + 1) * kUnitRows, qp.t_q) - 1;
+  int n = qp.kv_end[qp.nqc - 1];
+  for (int c = 0; c < qp.nqc; ++c)
+    if (last < qp.row_end[c]) { n = qp.kv_end[c]; break; }
+  return (n + wfk::kBN - 1) / wfk::kBN;
+}
+
+// Every split must own at least one key tile of every unit.
+int max_splits(const QueryPlan& qp) {
+  int m = kMaxSplits;
+  for (int pr = 0; pr < num_pairs(qp); ++pr) m = std::min(m, unit_tiles(qp, pr));
+  return std::max(m, 1);
+}
+
+size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+// part_o: fp32 [S][T_q][H][D], then part_lse: fp32 [S][H][T_q].
+size_t split_workspace_bytes(const QueryPlan& qp, int H, int D, int S) {
+  if (S <= 1) return 0;
+  const size_t rows = static_cast<size_t>(S) * qp.t_q * H;
+  return align256(rows * D * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+// Key splits per unit, from how full the last wave of CTAs is.  With U units on G SMs (one CTA
+// per SM) a single pass fills (U/G) / ceil(U/G) of the SM-time; S splits fill
+// (S U/G) / ceil(S U/G) but pay S - 1 more prologues per unit and a merge pass.  Split only a
+// grid shorter than two waves whose last wave is less than 80 % full, into the fewest splits
+// that fill 90 %.  (Measured on one Wave-Parallelism rank's call, 228 units on 148 SMs:
+// S = 1, 2, 3, 5, 6, 16 -> 1.18, 1.22, 1.16, 1.16, 1.35, 1.53 ms: tail waves cost about what
+// this fill predicts, and further splits only add overhead.)
+int choose_splits(const QueryPlan& qp, int H, int num_sms) {
+  const int64_t units = static_cast<int64_t>(num_pairs(qp)) * H;
+  auto fill = [&](int S) {
+    const double waves = static_cast<double>(units) * S / num_sms;
+    return waves / std::ceil(waves);
+  };
+  if (units >= 2 * static_cast<int64_t>(num_sms) || fill(1) >= 0.8) return 1;
+  const int cap = max_splits(qp);
+  for (int S = 2; S <= cap; ++S)
+    if (fill(S) >= 0.9) return S;
+  return 1;
+}
+
+// A validated attention launch.
+struct AttnLaunch {
+  alignas(64) wfk::AttnParams p;
+  QueryPlan qp;
+  DeviceState* d = nullptr;
+  int D = 0;
+  bool use_pair = false;
+  float* lse_out = nullptr;   // the caller's lse (written by the combine pass when split)
+};
+
+int prepare_attention(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* page_table_row,
+                      const wf_wavefront_t* wf, float scale, void* out, float* lse_or_null,
+                      AttnLaunch* L) {
+  int rc = validate_pool(kv_pages);
+  if (rc) return rc;
+  int t_kv = 0;
+  rc = validate_wavefront(wf, kv_pages, &t_kv);
+  if (rc) return rc;
+  if (wf->num_ctx_chunks >= wf->num_chunks) return WF_ERR_SHAPE;   // no query chunk
+  if (!(scale > 0.f) || !std::isfinite(scale)) return WF_ERR_INVALID_ARG;
+  rc = query_plan(wf, &L->qp);
+  if (rc) return rc;
+  wfk::AttnParams& p = L->p;
+  std::memset(&p, 0, sizeof(p));
+  const int t_q = L->qp.t_q;
+  if (t_q == 0) return WF_OK;                                        // nothing to compute
+  if (q == nullptr || out == nullptr || page_table_row == nullptr || !aligned16(q) ||
+      !aligned16(out) || (lse_or_null != nullptr && (reinterpret_cast<uintptr_t>(lse_or_null) & 3u)))
+    return WF_ERR_INVALID_ARG;
+  rc = device_state(&L->d);
+  if (rc) return rc;
+
+  const int H = kv_pages->num_heads, D = kv_pages->head_dim, ps = kv_pages->page_size;
+  static_assert(alignof(wfk::AttnParams) >= 64, "tensor maps need 64-byte alignment");
+  L->D = D;
+  // CTA pairs run head_dim 128; a box never crosses a page or a tile edge
+  L->use_pair = (D == 128) && WF_ATTN_PAIR;
+  const int box_rows = gcd_int(ps, L->use_pair ? 64 : wfk::kBN);
+  const int box_rows_v = gcd_int(ps, L->use_pair ? wfk::kPairBN : wfk::kBN);
+  const int64_t total_rows = static_cast<int64_t>(kv_pages->num_pages) * ps;
+  if (!encode_rows(&p.tm_q, q, D, H, t_q, wfk::kBM, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
+      !encode_rows(&p.tm_k, kv_pages->k_pool, D, H, total_rows, box_rows,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+      !encode_rows(&p.tm_v, kv_pages->v_pool, D, H, total_rows, box_rows_v,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+    return WF_ERR_CUDA;
+  p.box_rows_v = box_rows_v;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse_or_null;
+  L->lse_out = lse_or_null;
+  p.page_table = page_table_row;
+  p.status = L->d->status;
+  p.grid_abort = L->d->abort_word;
+  p.T_q = t_q;
+  p.H = H;
+  p.num_pages = kv_pages->num_pages;
+  p.page_size = ps;
+  p.total_rows = static_cast<int>(total_rows);
+  p.box_rows = box_rows;
+  p.n_pairs = num_pairs(L->qp);
+  p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.nqc = L->qp.nqc;
+  for (int c = 0; c < L->qp.nqc; ++c) {
+    p.qc_row_end[c] = L->qp.row_end[c];
+    p.qc_kv_end[c] = L->qp.kv_end[c];
+  }
+  p.n_splits = 1;
+  if (static_cast<int64_t>(p.n_pairs) * H * kMaxSplits * 2 > INT32_MAX) return WF_ERR_SHAPE;
+  return WF_OK;
+}
+
+// Point the launch at a workspace holding S partial results.
+void set_split_buffers(AttnLaunch* L, int S, void* workspace) {
+  const size_t rows = static_cast<size_t>(S) * L->qp.t_q * L->p.H;
+  L->p.n_splits = S;
+  L->p.part_o = static_cast<float*>(workspace);
+  L->p.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                           align256(rows * L->D * sizeof(float)));
+}
+
+int launch_attention(AttnLaunch* L, cudaStream_t s) {
+  wfk::AttnParams& p = L->p;
+  p.launch_id = g_launch_counter.fetch_add(1);
+  if (p.launch_id == 0) p.launch_id = g_launch_counter.fetch_add(1);
+  const int64_t grid = static_cast<int64_t>(p.n_pairs) * p.H * p.n_splits;
+  if (L->use_pair)
+    wfk::wf_attn_pair_kernel<<<static_cast<unsigned>(2 * grid), wfk::kPairThreads,
+                               wfk::PairSmem::ALLOC, s>>>(p);
+  else if (L->D == 128)
+    wfk::wf_attn_fwd_kernel<128><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
+                                   wfk::AttnSmem<128>::ALLOC, s>>>(p);
+  else
+    wfk::wf_attn_fwd_kernel<64><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
+                                  wfk::AttnSmem<64>::ALLOC, s>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return WF_ERR_CUDA;
+  if (p.n_splits > 1) {
+    const int64_t threads = static_cast<int64_t>(p.T_q) * p.H * 32;
+    const unsigned blocks =
+        static_cast<unsigned>((threads + wfk::kCombineThreads - 1) / wfk::kCombineThreads);
+    if (L->D == 128)
+      wfk::wf_combine_kernel<128><<<blocks, wfk::kCombineThreads, 0, s>>>(
+          p.part_o, p.part_lse, p.n_splits, p.T_q, p.H, p.out, L->lse_out);
+    else
+      wfk::wf_combine_kernel<64><<<blocks, wfk::kCombineThreads, 0, s>>>(
+          p.part_o, p.part_lse, p.n_splits, p.T_q, p.H, p.out, L->lse_out);
+    if (cudaGetLastError() != cudaSuccess) return WF_ERR_CUDA;
+  }
+  return WF_OK;
+}
+
+
 // One CTA waits on a barrier nobody arrives on; the bounded wait must give up, record
 // WF_ERR_TIMEOUT and return.
 __global__ void wf_selftest_timeout_kernel(int* status, unsigned* grid_abort, unsigned launch_id,
@@ -232,76 +423,45 @@ int wf_kv_append(const wf_kv_pool_t* pool, int layer, int chunk, const void* k, 
 int wf_attn_forward(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* page_table_row,
                     const wf_wavefront_t* wf, float scale, void* out, float* lse_or_null,
                     wf_stream_t stream) {
-  int rc = validate_pool(kv_pages);
-  if (rc) return rc;
-  int t_kv = 0;
-  rc = validate_wavefront(wf, kv_pages, &t_kv);
-  if (rc) return rc;
-  if (wf->num_ctx_chunks >= wf->num_chunks) return WF_ERR_SHAPE;   // no query chunk
-  if (!(scale > 0.f) || !std::isfinite(scale)) return WF_ERR_INVALID_ARG;
-  const int t_ctx = wf->chunk_offsets[wf->num_ctx_chunks];
-  const int t_q = t_kv - t_ctx;
-  if (t_q == 0) return WF_OK;
-  if (q == nullptr || out == nullptr || page_table_row == nullptr || !aligned16(q) ||
-      !aligned16(out) || (lse_or_null != nullptr && (reinterpret_cast<uintptr_t>(lse_or_null) & 3u)))
-    return WF_ERR_INVALID_ARG;
-  DeviceState* d = nullptr;
-  rc = device_state(&d);
-  if (rc) return rc;
+  AttnLaunch L;
+  const int rc = prepare_attention(q, kv_pages, page_table_row, wf, scale, out, lse_or_null, &L);
+  if (rc || L.p.T_q == 0) return rc;
+  return launch_attention(&L, reinterpret_cast<cudaStream_t>(stream));
+}
 
-  const int H = kv_pages->num_heads, D = kv_pages->head_dim, ps = kv_pages->page_size;
-  static_assert(alignof(wfk::AttnParams) >= 64, "tensor maps need 64-byte alignment");
-  wfk::AttnParams p;
-  std::memset(&p, 0, sizeof(p));
-  // CTA pairs run head_dim 128; a box never crosses a page or a tile edge
-  const bool use_pair = (D == 128) && WF_ATTN_PAIR;
-  const int box_rows = gcd_int(ps, use_pair ? 64 : wfk::kBN);
-  const int box_rows_v = gcd_int(ps, use_pair ? wfk::kPairBN : wfk::kBN);
-  const int64_t total_rows = static_cast<int64_t>(kv_pages->num_pages) * ps;
-  if (!encode_rows(&p.tm_q, q, D, H, t_q, wfk::kBM, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
-      !encode_rows(&p.tm_k, kv_pages->k_pool, D, H, total_rows, box_rows,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
-      !encode_rows(&p.tm_v, kv_pages->v_pool, D, H, total_rows, box_rows_v,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
-    return WF_ERR_CUDA;
-  p.box_rows_v = box_rows_v;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse_or_null;
-  p.page_table = page_table_row;
-  p.status = d->status;
-  p.grid_abort = d->abort_word;
-  p.T_q = t_q;
-  p.H = H;
-  p.num_pages = kv_pages->num_pages;
-  p.page_size = ps;
-  p.total_rows = static_cast<int>(total_rows);
-  p.box_rows = box_rows;
-  p.n_pairs = (t_q + wfk::kNQT * wfk::kBM - 1) / (wfk::kNQT * wfk::kBM);
-  p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  p.launch_id = g_launch_counter.fetch_add(1);
-  if (p.launch_id == 0) p.launch_id = g_launch_counter.fetch_add(1);
-  int nqc = 0;
-  for (int c = wf->num_ctx_chunks; c < wf->num_chunks; ++c) {
-    if (wf->chunk_offsets[c + 1] == wf->chunk_offsets[c]) continue;   // empty chunk: no rows
-    p.qc_row_end[nqc] = wf->chunk_offsets[c + 1] - t_ctx;
-    p.qc_kv_end[nqc] = wf->chunk_offsets[c + 1];
-    ++nqc;
+size_t wf_attn_workspace_size(const wf_wavefront_t* wf, int num_heads, int head_dim, int splits) {
+  QueryPlan qp;
+  if (wf == nullptr || num_heads < 1 || (head_dim != 64 && head_dim != 128) || splits < 0 ||
+      query_plan(wf, &qp) != WF_OK || qp.t_q == 0)
+    return 0;
+  int S = splits;
+  if (S == 0) {
+    DeviceState* d = nullptr;
+    if (device_state(&d) != WF_OK) return 0;
+    S = choose_splits(qp, num_heads, d->num_sms);
   }
-  p.nqc = nqc;
+  S = std::min(S, max_splits(qp));
+  return split_workspace_bytes(qp, num_heads, head_dim, S);
+}
 
-  const int64_t grid = static_cast<int64_t>(p.n_pairs) * H;
-  if (2 * grid > INT32_MAX) return WF_ERR_SHAPE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (use_pair)
-    wfk::wf_attn_pair_kernel<<<static_cast<unsigned>(2 * grid), wfk::kPairThreads,
-                               wfk::PairSmem::ALLOC, s>>>(p);
-  else if (D == 128)
-    wfk::wf_attn_fwd_kernel<128><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
-                                   wfk::AttnSmem<128>::ALLOC, s>>>(p);
-  else
-    wfk::wf_attn_fwd_kernel<64><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
-                                  wfk::AttnSmem<64>::ALLOC, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+int wf_attn_forward_split(const void* q, const wf_kv_pool_t* kv_pages,
+                          const int32_t* page_table_row, const wf_wavefront_t* wf, float scale,
+                          void* out, float* lse_or_null, int splits, void* workspace,
+                          size_t workspace_bytes, wf_stream_t stream) {
+  if (splits < 0) return WF_ERR_INVALID_ARG;
+  AttnLaunch L;
+  const int rc = prepare_attention(q, kv_pages, page_table_row, wf, scale, out, lse_or_null, &L);
+  if (rc || L.p.T_q == 0) return rc;
+  int S = splits > 0 ? splits : choose_splits(L.qp, L.p.H, L.d->num_sms);
+  S = std::min(S, max_splits(L.qp));
+  if (L.use_pair) S = 1;                       // the CTA-pair kernel has no key splits
+  if (S > 1) {
+    const size_t need = split_workspace_bytes(L.qp, L.p.H, L.D, S);
+    if (workspace == nullptr || !aligned16(workspace)) return WF_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return WF_ERR_CAPACITY;
+    set_split_buffers(&L, S, workspace);
+  }
+  return launch_attention(&L, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int wf_selftest_timeout(unsigned timeout_us, wf_stream_t stream) {

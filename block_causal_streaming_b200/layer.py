@@ -45,6 +45,7 @@ class WavefrontLayer:
                                        page_tables.shape[1])
         self.chunk_offsets = list(chunk_offsets)
         self.num_ctx_chunks = int(num_ctx_chunks)
+        self._workspace: Optional[torch.Tensor] = None   # split-KV partial results
 
     @property
     def t_q(self) -> int:
@@ -62,8 +63,22 @@ class WavefrontLayer:
             self.append(c, k_all[a:b], v_all[a:b], stream)
 
     def forward(self, q: torch.Tensor, out: torch.Tensor, scale: Optional[float] = None,
-                lse: Optional[torch.Tensor] = None, stream=None) -> None:
+                lse: Optional[torch.Tensor] = None, stream=None,
+                splits: Optional[int] = None) -> None:
+        """Attention of ``q`` over this layer's pages.  ``splits`` None: wf_attn_forward; an int:
+        wf_attn_forward_split with that many key splits (0: the library's choice), with a
+        workspace this layer allocates once and reuses."""
         if scale is None:
             scale = 1.0 / math.sqrt(self.pool.head_dim)
-        _abi.attn_forward(q, self.pool.k, self.pool.v, self.page_tables[self.layer], self.desc,
-                          scale, out, lse, stream)
+        if splits is None:
+            _abi.attn_forward(q, self.pool.k, self.pool.v, self.page_tables[self.layer],
+                              self.desc, scale, out, lse, stream)
+            return
+        need = _abi.attn_workspace_size(self.desc, self.pool.heads, self.pool.head_dim, splits)
+        ws = None
+        if need > 0:
+            if self._workspace is None or self._workspace.numel() < need:
+                self._workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+            ws = self._workspace
+        _abi.attn_forward_split(q, self.pool.k, self.pool.v, self.page_tables[self.layer],
+                                self.desc, scale, out, splits, ws, lse, stream)

@@ -120,6 +120,14 @@ WAN14B = Workload("wan14b_6ctx+5x4680_h40_d128_ps128", heads=40, head_dim=128,
 
 CONFIGS = {1: TINY, 2: WAN13B_5STEP, 3: WAN13B_4STEP, 4: WAN13B_ROUND30, 5: WAN14B}
 
+# One Wave-Parallelism rank's call: the critical consumer's single query chunk against a context
+# of 7 earlier chunks (8 chunks visible; project page, "02 Interactive pipeline", "Inside one
+# diffusion tick").  Seed 5; otherwise the 1.3B shapes above.
+WP_RANK0 = Workload("wp_rank0_7ctx+1x4680_h12_d128", heads=12, head_dim=128,
+                    ctx_lens=(CHUNK_TOKENS,) * 7, active_lens=(CHUNK_TOKENS,),
+                    active_stages=(1000,), page_size=64, value_scale=0.5, seed=5,
+                    page_order="perm")
+
 
 def small_case(name: str, heads: int, head_dim: int, ctx_lens, active_lens, page_size: int,
                seed: int, value_scale: float = 1.0, k_mean_offset: bool = False,

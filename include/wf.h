@@ -131,6 +131,36 @@ int wf_attn_forward(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* 
                     wf_stream_t stream);
 
 /*
+ * wf_attn_forward_split -- the same attention with every unit's key range split over several CTAs
+ * (split-KV), for wavefronts with too few query rows to fill the GPU -- one Wave-Parallelism
+ * rank's call, a single query chunk against a long prefix (project page, "02 Interactive
+ * pipeline", "Inside one diffusion tick": the critical consumer sees 8 chunks).  Each of the S
+ * CTAs of a unit computes a normalised partial output and log-sum-exp over its consecutive part
+ * of the unit's key tiles; a second kernel merges them (out = sum_s exp(lse_s - lse) O_s).
+ * Arguments and result as wf_attn_forward, plus:
+ *   splits           S >= 1 key splits per unit (capped at 16 and at the key tiles of the
+ *                    smallest unit), or 0 to let the library pick S from a model of the grid.
+ *   workspace        device memory, 16-byte aligned, caller-owned, at least
+ *                    wf_attn_workspace_size(wf, H, D, splits) bytes; may be null when that
+ *                    size is 0 (S = 1 runs exactly wf_attn_forward's single pass).
+ * Errors: as wf_attn_forward; WF_ERR_CAPACITY if workspace_bytes is too small; WF_ERR_INVALID_ARG
+ * for splits < 0 or a null/misaligned workspace that is needed.  Two launches on `stream`; the
+ * workspace must not be shared by calls that may run concurrently.
+ */
+int wf_attn_forward_split(const void* q, const wf_kv_pool_t* kv_pages,
+                          const int32_t* page_table_row, const wf_wavefront_t* wf, float scale,
+                          void* out, float* lse_or_null, int splits, void* workspace,
+                          size_t workspace_bytes, wf_stream_t stream);
+
+/*
+ * wf_attn_workspace_size -- bytes of workspace wf_attn_forward_split needs for this wavefront,
+ * head count, head_dim and `splits` (0: the library's choice on the current device):
+ * S * T_q * H * (D + 1) * 4 bytes (fp32 partial outputs and log-sum-exps, each rounded up to 256)
+ * when S > 1, else 0.  Also 0 for invalid arguments (the forward call then reports the error).
+ */
+size_t wf_attn_workspace_size(const wf_wavefront_t* wf, int num_heads, int head_dim, int splits);
+
+/*
  * wf_check_status -- synchronise `stream`, then return and clear the first error any kernel of
  * this library recorded on the current device since the last call (WF_OK if none).  A pending
  * CUDA error on the stream is returned as WF_ERR_CUDA.

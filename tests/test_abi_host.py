@@ -122,3 +122,39 @@ def test_valid_call_without_device_reports_no_device(abi):
     desc = abi.WavefrontDesc([0, 64, 128, 200], [0, 200, 1000], 1, 8)
     assert _attn(abi, _pool(abi), desc) == abi.WF_ERR_NO_DEVICE
     assert _append(abi, _pool(abi), desc) == abi.WF_ERR_NO_DEVICE
+
+
+def test_split_workspace_size_formula(abi):
+    """S * T_q * H * (D + 1) fp32 values, each array rounded up to 256 bytes; none for S = 1."""
+    desc = abi.WavefrontDesc([0, 4680, 9360], [0, 1000], 1, 200)     # T_q = 4680
+    for heads, d, s in ((12, 128, 4), (2, 64, 3), (40, 128, 16)):
+        rows = s * 4680 * heads
+        up = lambda n: (n + 255) // 256 * 256
+        assert abi.lib.wf_attn_workspace_size(ctypes.byref(desc.c), heads, d, s) == \
+            up(rows * d * 4) + up(rows * 4)
+    assert abi.lib.wf_attn_workspace_size(ctypes.byref(desc.c), 12, 128, 1) == 0
+    # capped at the key tiles of the smallest unit: 9360 keys = 74 tiles, cap 16
+    assert abi.lib.wf_attn_workspace_size(ctypes.byref(desc.c), 12, 128, 99) == \
+        abi.lib.wf_attn_workspace_size(ctypes.byref(desc.c), 12, 128, 16)
+    small = abi.WavefrontDesc([0, 100, 200], [0, 0], 1, 200)        # 200 keys: 2 tiles
+    assert abi.lib.wf_attn_workspace_size(ctypes.byref(small.c), 1, 128, 8) == \
+        abi.lib.wf_attn_workspace_size(ctypes.byref(small.c), 1, 128, 2)
+    # invalid arguments give 0 (the forward call reports the error)
+    assert abi.lib.wf_attn_workspace_size(ctypes.byref(desc.c), 12, 96, 4) == 0
+    assert abi.lib.wf_attn_workspace_size(ctypes.byref(desc.c), 0, 128, 4) == 0
+    assert abi.lib.wf_attn_workspace_size(ctypes.byref(desc.c), 12, 128, -1) == 0
+
+
+def test_split_validation_errors_without_a_gpu(abi):
+    ok_desc = abi.WavefrontDesc([0, 64, 128, 200], [0, 200, 1000], 1, 8)
+
+    def split(pool, desc, splits=2, ws=None, nbytes=0):
+        return abi.lib.wf_attn_forward_split(
+            FAKE, ctypes.byref(pool), ctypes.cast(ctypes.c_void_p(FAKE), ctypes.POINTER(ctypes.c_int32)),
+            ctypes.byref(desc.c), 0.1, FAKE, None, splits, ws, nbytes, None)
+    assert split(_pool(abi), ok_desc, splits=-1) == abi.WF_ERR_INVALID_ARG
+    assert split(_pool(abi, head_dim=96), ok_desc) == abi.WF_ERR_SHAPE
+    assert split(_pool(abi), abi.WavefrontDesc([0, 64, 128], [500, 200], 0, 8)) == \
+        abi.WF_ERR_STAGE_ORDER
+    empty = abi.WavefrontDesc([0, 64, 64], [0, 0], 1, 8)
+    assert split(_pool(abi), empty) == abi.WF_OK
