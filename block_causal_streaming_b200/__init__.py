@@ -17,6 +17,7 @@ _ABI_NAMES = (
     "WF_ERR_PAGE_OOB", "WF_ERR_TIMEOUT", "WF_ERR_CUDA", "WF_ERR_NO_DEVICE", "WF_MAX_CHUNKS",
     "WavefrontDesc", "WfError", "attn_forward", "check_status", "kv_append", "strerror",
     "selftest_timeout", "attn_forward_split", "attn_workspace_size",
+    "attn_forward_split_noalloc",
 )
 __all__ = list(_ABI_NAMES)
 

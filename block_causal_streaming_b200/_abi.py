@@ -26,7 +26,8 @@ WF_MAX_CHUNKS = 64
 
 # Every symbol include/wf.h declares (checked by the CPU tests).
 EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror", "wf_version",
-            "wf_selftest_timeout", "wf_attn_forward_split", "wf_attn_workspace_size")
+            "wf_selftest_timeout", "wf_attn_forward_split", "wf_attn_workspace_size",
+            "wf_attn_forward_split_noalloc")
 
 
 class WfError(RuntimeError):
@@ -75,6 +76,11 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
                                           ctypes.POINTER(ctypes.c_float), i32, vp,
                                           ctypes.c_size_t, vp]
     lib.wf_attn_forward_split.restype = i32
+    lib.wf_attn_forward_split_noalloc.argtypes = [vp, ctypes.POINTER(KvPool),
+                                                  ctypes.POINTER(ctypes.c_int32),
+                                                  ctypes.POINTER(Wavefront), ctypes.c_float, vp,
+                                                  ctypes.POINTER(ctypes.c_float), i32, vp]
+    lib.wf_attn_forward_split_noalloc.restype = i32
     lib.wf_attn_workspace_size.argtypes = [ctypes.POINTER(Wavefront), i32, i32, i32]
     lib.wf_attn_workspace_size.restype = ctypes.c_size_t
     return lib
@@ -191,6 +197,27 @@ def attn_forward_split(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, sca
         _stream_handle(stream))
     if rc != WF_OK:
         raise WfError(rc, "wf_attn_forward_split")
+
+
+def attn_forward_split_noalloc(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc,
+                               scale: float, out, splits: int = 0, lse=None, stream=None) -> None:
+    """wf_attn_forward_split_noalloc: attn_forward_split with the library's static scratch
+    instead of a workspace (calls on one device must be ordered on one stream)."""
+    for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
+                    (page_table_row, "page_table_row", "i32"), (out, "out", "bf16")):
+        _check_tensor(t, n, d)
+    if lse is not None:
+        _check_tensor(lse, "lse", "f32")
+    pool = _pool_struct(k_pool, v_pool)
+    rc = lib.wf_attn_forward_split_noalloc(
+        q.data_ptr(), ctypes.byref(pool),
+        ctypes.cast(ctypes.c_void_p(page_table_row.data_ptr()), ctypes.POINTER(ctypes.c_int32)),
+        ctypes.byref(wf.c), float(scale), out.data_ptr(),
+        ctypes.cast(ctypes.c_void_p(lse.data_ptr()), ctypes.POINTER(ctypes.c_float))
+        if lse is not None else None,
+        int(splits), _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_attn_forward_split_noalloc")
 
 
 def selftest_timeout(timeout_us: int, stream=None) -> None:

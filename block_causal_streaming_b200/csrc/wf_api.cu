@@ -28,6 +28,12 @@ __device__ unsigned g_wf_abort = 0;
 #define WF_ATTN_PAIR 0
 #endif
 
+// Scratch of wf_attn_forward_split_noalloc: one static array per device, so that entry point
+// needs no allocation.  96 MiB holds the partial results of 3 key splits of a 4680-row, 12-head,
+// head_dim-128 call (3 x 4680 x 12 x 129 x 4 B = 86.9 MB); larger plans are rejected.
+constexpr size_t kScratchBytes = size_t(96) << 20;
+__device__ __align__(256) unsigned char g_wf_scratch[kScratchBytes];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -241,6 +247,27 @@ int choose_splits(const QueryPlan& qp, int H, int num_sms) {
   for (int S = 2; S <= cap; ++S)
     if (fill(S) >= 0.9) return S;
   return 1;
+}
+
+// Device address of g_wf_scratch on the current device, looked up once per device.
+void* g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+int scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return WF_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr &&
+      cudaGetSymbolAddress(&g_scratch_addr[dev], g_wf_scratch) != cudaSuccess) {
+    cudaGetLastError();
+    g_scratch_addr[dev] = nullptr;
+    return WF_ERR_CUDA;
+  }
+  *out = g_scratch_addr[dev];
+  return WF_OK;
 }
 
 // A validated attention launch.
@@ -460,6 +487,27 @@ int wf_attn_forward_split(const void* q, const wf_kv_pool_t* kv_pages,
     if (workspace == nullptr || !aligned16(workspace)) return WF_ERR_INVALID_ARG;
     if (workspace_bytes < need) return WF_ERR_CAPACITY;
     set_split_buffers(&L, S, workspace);
+  }
+  return launch_attention(&L, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int wf_attn_forward_split_noalloc(const void* q, const wf_kv_pool_t* kv_pages,
+                                  const int32_t* page_table_row, const wf_wavefront_t* wf,
+                                  float scale, void* out, float* lse_or_null, int splits,
+                                  wf_stream_t stream) {
+  if (splits < 0) return WF_ERR_INVALID_ARG;
+  AttnLaunch L;
+  int rc = prepare_attention(q, kv_pages, page_table_row, wf, scale, out, lse_or_null, &L);
+  if (rc || L.p.T_q == 0) return rc;
+  int S = splits > 0 ? splits : choose_splits(L.qp, L.p.H, L.d->num_sms);
+  S = std::min(S, max_splits(L.qp));
+  if (L.use_pair) S = 1;
+  if (S > 1) {
+    if (split_workspace_bytes(L.qp, L.p.H, L.D, S) > kScratchBytes) return WF_ERR_CAPACITY;
+    void* scratch = nullptr;
+    rc = scratch_address(&scratch);
+    if (rc) return rc;
+    set_split_buffers(&L, S, scratch);
   }
   return launch_attention(&L, reinterpret_cast<cudaStream_t>(stream));
 }

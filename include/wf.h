@@ -153,6 +153,23 @@ int wf_attn_forward_split(const void* q, const wf_kv_pool_t* kv_pages,
                           size_t workspace_bytes, wf_stream_t stream);
 
 /*
+ * wf_attn_forward_split_noalloc -- wf_attn_forward_split without a caller workspace: the partial
+ * results go to a static 96 MiB (100 663 296-byte) array the library keeps in device memory, one
+ * per device, so the call allocates nothing.  No counterpart on the pages: it exists for callers
+ * that cannot hand over device memory.  Arguments and result as wf_attn_forward_split without
+ * `workspace` / `workspace_bytes`; WF_ERR_CAPACITY when the plan needs more than the 96 MiB
+ * (S * T_q * H * (D + 1) * 4 bytes; pass a smaller `splits` or use wf_attn_forward_split).
+ * Sharing: every call on a device uses the same array.  Calls that may run at the same time --
+ * on different streams of one device, or from several host threads without ordering -- race on
+ * it and may return wrong results; order them on one stream (the array is only read by the
+ * merge kernel of the same call, which runs after the attention kernel on that stream).
+ */
+int wf_attn_forward_split_noalloc(const void* q, const wf_kv_pool_t* kv_pages,
+                                  const int32_t* page_table_row, const wf_wavefront_t* wf,
+                                  float scale, void* out, float* lse_or_null, int splits,
+                                  wf_stream_t stream);
+
+/*
  * wf_attn_workspace_size -- bytes of workspace wf_attn_forward_split needs for this wavefront,
  * head count, head_dim and `splits` (0: the library's choice on the current device):
  * S * T_q * H * (D + 1) * 4 bytes (fp32 partial outputs and log-sum-exps, each rounded up to 256)
