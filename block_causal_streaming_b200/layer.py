@@ -46,6 +46,7 @@ class WavefrontLayer:
         self.chunk_offsets = list(chunk_offsets)
         self.num_ctx_chunks = int(num_ctx_chunks)
         self._workspace: Optional[torch.Tensor] = None   # split-KV partial results
+        self._ws_bytes: dict = {}                          # workspace bytes per `splits`
 
     @property
     def t_q(self) -> int:
@@ -74,7 +75,11 @@ class WavefrontLayer:
             _abi.attn_forward(q, self.pool.k, self.pool.v, self.page_tables[self.layer],
                               self.desc, scale, out, lse, stream)
             return
-        need = _abi.attn_workspace_size(self.desc, self.pool.heads, self.pool.head_dim, splits)
+        need = self._ws_bytes.get(splits)
+        if need is None:
+            need = _abi.attn_workspace_size(self.desc, self.pool.heads, self.pool.head_dim,
+                                            splits)
+            self._ws_bytes[splits] = need
         ws = None
         if need > 0:
             if self._workspace is None or self._workspace.numel() < need:
