@@ -5,7 +5,10 @@ The product is the C-ABI library ``libwf_b200.so`` (declared in ``include/wf.h``
 * ``wf_kv_append``    -- publish one chunk's layer-wise K/V into fixed-size pages;
 * ``wf_attn_forward`` -- one block-causal attention over every chunk of the wavefront, one launch;
 * ``wf_attn_forward_split`` -- the same with each unit's keys split over several CTAs and merged,
-  for wavefronts with few query rows (one Wave-Parallelism rank's chunk against its prefix).
+  for wavefronts with few query rows (one Wave-Parallelism rank's chunk against its prefix);
+* ``wf_kv_append_publish`` / ``wf_attn_forward_published`` -- one-way publication of a chunk's
+  K/V into other GPUs' pools with a generation flag, and attention that waits for the flags
+  (:mod:`.wave` maps the peers' pools between processes).
 
 This package is its thin Python binding (ctypes, argument marshalling only), a small helper that
 owns the paged pools of one layer (:mod:`.layer`) and the seeded synthetic workloads
@@ -17,7 +20,8 @@ _ABI_NAMES = (
     "WF_ERR_PAGE_OOB", "WF_ERR_TIMEOUT", "WF_ERR_CUDA", "WF_ERR_NO_DEVICE", "WF_MAX_CHUNKS",
     "WavefrontDesc", "WfError", "attn_forward", "check_status", "kv_append", "strerror",
     "selftest_timeout", "attn_forward_split", "attn_workspace_size",
-    "attn_forward_split_noalloc",
+    "attn_forward_split_noalloc", "kv_append_publish", "attn_forward_published", "ipc_export",
+    "ipc_import", "ipc_close", "PoolDst",
 )
 __all__ = list(_ABI_NAMES)
 

@@ -27,13 +27,20 @@ WF_MAX_CHUNKS = 64
 # Every symbol include/wf.h declares (checked by the CPU tests).
 EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror", "wf_version",
             "wf_selftest_timeout", "wf_attn_forward_split", "wf_attn_workspace_size",
-            "wf_attn_forward_split_noalloc")
+            "wf_attn_forward_split_noalloc", "wf_kv_append_publish", "wf_attn_forward_published",
+            "wf_ipc_export", "wf_ipc_import", "wf_ipc_close")
 
 
 class WfError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
         super().__init__(f"{what}: {strerror(code)}")
+
+
+class PoolDst(ctypes.Structure):
+    """wf_pool_dst_t: a destination pool (usually another GPU's, mapped by ipc_import)."""
+    _fields_ = [("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p),
+                ("flags", ctypes.c_void_p)]
 
 
 class KvPool(ctypes.Structure):
@@ -81,6 +88,22 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
                                                   ctypes.POINTER(Wavefront), ctypes.c_float, vp,
                                                   ctypes.POINTER(ctypes.c_float), i32, vp]
     lib.wf_attn_forward_split_noalloc.restype = i32
+    lib.wf_kv_append_publish.argtypes = [ctypes.POINTER(KvPool), vp, ctypes.POINTER(PoolDst),
+                                         i32, i32, i32, vp, vp, ctypes.POINTER(ctypes.c_int32),
+                                         ctypes.POINTER(Wavefront), ctypes.c_uint32, vp]
+    lib.wf_kv_append_publish.restype = i32
+    lib.wf_attn_forward_published.argtypes = [vp, ctypes.POINTER(KvPool),
+                                              ctypes.POINTER(ctypes.c_int32),
+                                              ctypes.POINTER(Wavefront), ctypes.c_float, vp,
+                                              ctypes.POINTER(ctypes.c_float), vp,
+                                              ctypes.c_uint32, i32, vp, ctypes.c_size_t, vp]
+    lib.wf_attn_forward_published.restype = i32
+    lib.wf_ipc_export.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_size_t)]
+    lib.wf_ipc_export.restype = i32
+    lib.wf_ipc_import.argtypes = [vp, ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p)]
+    lib.wf_ipc_import.restype = i32
+    lib.wf_ipc_close.argtypes = [vp]
+    lib.wf_ipc_close.restype = i32
     lib.wf_attn_workspace_size.argtypes = [ctypes.POINTER(Wavefront), i32, i32, i32]
     lib.wf_attn_workspace_size.restype = ctypes.c_size_t
     return lib
@@ -123,9 +146,10 @@ def _stream_handle(stream) -> Optional[int]:
 
 def _check_tensor(t, name: str, dtype_name: str):
     import torch
-    want = {"bf16": torch.bfloat16, "i32": torch.int32, "f32": torch.float32}[dtype_name]
-    if t.dtype != want:
-        raise TypeError(f"{name}: expected {want}, got {t.dtype}")
+    want = {"bf16": (torch.bfloat16,), "i32": (torch.int32,), "f32": (torch.float32,),
+            "u32": (torch.int32, torch.uint32)}[dtype_name]      # flag words: any 32-bit int
+    if t.dtype not in want:
+        raise TypeError(f"{name}: expected {want[0]}, got {t.dtype}")
     if not t.is_cuda:
         raise ValueError(f"{name}: expected a CUDA tensor")
     if not t.is_contiguous():
@@ -218,6 +242,87 @@ def attn_forward_split_noalloc(q, k_pool, v_pool, page_table_row, wf: WavefrontD
         int(splits), _stream_handle(stream))
     if rc != WF_OK:
         raise WfError(rc, "wf_attn_forward_split_noalloc")
+
+
+def kv_append_publish(k_pool, v_pool, flags, peers, layer: int, chunk: int, k, v, page_table,
+                      wf: WavefrontDesc, generation: int, stream=None) -> None:
+    """wf_kv_append_publish: append one chunk into this pool and every peer pool, then raise the
+    chunk's flag to ``generation`` here (``flags``: device uint32 [layers, WF_MAX_CHUNKS] or
+    None) and in every peer.  ``peers``: sequence of (k_pool_ptr, v_pool_ptr, flags_ptr)."""
+    for t, n, d in ((k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
+                    (page_table, "page_table", "i32")):
+        _check_tensor(t, n, d)
+    if k.numel() > 0:
+        _check_tensor(k, "k", "bf16")
+        _check_tensor(v, "v", "bf16")
+    if flags is not None:
+        _check_tensor(flags, "flags", "u32")
+    arr = (PoolDst * max(1, len(peers)))(*[PoolDst(int(a), int(b), int(c) if c else None)
+                                          for a, b, c in peers])
+    pool = _pool_struct(k_pool, v_pool)
+    rc = lib.wf_kv_append_publish(
+        ctypes.byref(pool), flags.data_ptr() if flags is not None else None, arr, len(peers),
+        int(layer), int(chunk), k.data_ptr() if k.numel() else None,
+        v.data_ptr() if v.numel() else None,
+        ctypes.cast(ctypes.c_void_p(page_table.data_ptr()), ctypes.POINTER(ctypes.c_int32)),
+        ctypes.byref(wf.c), int(generation) & 0xFFFFFFFF, _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_kv_append_publish")
+
+
+def attn_forward_published(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: float,
+                           out, flags_row, generation: int, splits: int = 0, workspace=None,
+                           lse=None, stream=None) -> None:
+    """wf_attn_forward_published: attn_forward_split that waits, chunk by chunk, for the
+    publication flags in ``flags_row`` (device uint32 [WF_MAX_CHUNKS]) to reach ``generation``."""
+    for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
+                    (page_table_row, "page_table_row", "i32"), (out, "out", "bf16"),
+                    (flags_row, "flags_row", "u32")):
+        _check_tensor(t, n, d)
+    if lse is not None:
+        _check_tensor(lse, "lse", "f32")
+    pool = _pool_struct(k_pool, v_pool)
+    rc = lib.wf_attn_forward_published(
+        q.data_ptr(), ctypes.byref(pool),
+        ctypes.cast(ctypes.c_void_p(page_table_row.data_ptr()), ctypes.POINTER(ctypes.c_int32)),
+        ctypes.byref(wf.c), float(scale), out.data_ptr(),
+        ctypes.cast(ctypes.c_void_p(lse.data_ptr()), ctypes.POINTER(ctypes.c_float))
+        if lse is not None else None,
+        flags_row.data_ptr(), int(generation) & 0xFFFFFFFF, int(splits),
+        workspace.data_ptr() if workspace is not None else None,
+        workspace.numel() * workspace.element_size() if workspace is not None else 0,
+        _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_attn_forward_published")
+
+
+def ipc_export(device_ptr: int):
+    """wf_ipc_export: (64-byte IPC handle of the allocation holding ``device_ptr``, offset)."""
+    buf = ctypes.create_string_buffer(64)
+    off = ctypes.c_size_t()
+    rc = lib.wf_ipc_export(ctypes.c_void_p(int(device_ptr)), buf, ctypes.byref(off))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_ipc_export")
+    return buf.raw, int(off.value)
+
+
+def ipc_import(exported) -> int:
+    """wf_ipc_import: map another process's (handle, offset); returns the device pointer here."""
+    handle, offset = exported
+    if len(handle) != 64:
+        raise ValueError("an IPC handle has 64 bytes")
+    out = ctypes.c_void_p()
+    rc = lib.wf_ipc_import(ctypes.create_string_buffer(handle, 64), int(offset),
+                           ctypes.byref(out))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_ipc_import")
+    return int(out.value)
+
+
+def ipc_close(device_ptr: int) -> None:
+    rc = lib.wf_ipc_close(ctypes.c_void_p(int(device_ptr)))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_ipc_close")
 
 
 def selftest_timeout(timeout_us: int, stream=None) -> None:

@@ -97,6 +97,13 @@ struct AttnParams {
   int n_splits;
   float* part_o;                    // fp32 [n_splits][T_q][H][D]
   float* part_lse;                  // fp32 [n_splits][H][T_q], natural log; -inf: no key seen
+  // Published chunks (one-way K/V publication between GPUs): with flags != null the keys of
+  // chunk c are loaded only after flags[c] has reached flag_gen.  chunk_end[c]: exclusive end
+  // token of chunk c in the logical key order.
+  const unsigned* flags;
+  unsigned flag_gen;
+  int nchunks;
+  int chunk_end[kMaxQChunks];
 };
 
 __device__ __forceinline__ int kv_end_of_row(const AttnParams& p, int r) {
@@ -162,7 +169,9 @@ struct AttnSmem {
   static_assert(ALLOC <= 227u * 1024u, "shared memory per CTA exceeds 227 KB");
 };
 
-template <int D>
+// kWaitPublished: wait for the publication flags of the chunks (AttnParams::flags) before
+// loading their keys; a separate instantiation so the plain kernel carries none of that code.
+template <int D, bool kWaitPublished = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     wf_attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   using L = AttnSmem<D>;
@@ -325,56 +334,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // ------------------------------------------------------------------------- epilogue
       if (ok)
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_O + q), (nk - 1) & 1, w));
-      if (ok && p.n_splits > 1) {
-        // partial result of this key split: O / l in fp32 and its log-sum-exp (-inf, O = 0 if
-        // no key of this split is visible to the row)
+      if (ok) {
+        // O / l: bf16 into `out`, or -- for one key split of a unit -- fp32 into the partials,
+        // with O = 0 and lse = -inf when no key of the split is visible to the row.
         tc_fence_after();
+        const bool part = p.n_splits > 1;
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
         const bool live = row_g < p.T_q;
-        float* const prow =
-            p.part_o + ((static_cast<size_t>(split) * p.T_q + row_g) * p.H + head) * D;
-  #pragma unroll
+        const size_t orow = static_cast<size_t>(row_g) * p.H + head;
+        const size_t prow = static_cast<size_t>(split) * p.T_q * p.H + orow;
+  #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
           tmem_ld32(tO + 32u * c, r);
           tmem_wait_ld();
-          if (live) {
-            float4* dst = reinterpret_cast<float4*>(prow + 32 * c);
+          if (live && part) {
+            float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + 32 * c);
   #pragma unroll
             for (int i = 0; i < 8; ++i)
               dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv_l,
                                    __uint_as_float(r[4 * i + 1]) * inv_l,
                                    __uint_as_float(r[4 * i + 2]) * inv_l,
                                    __uint_as_float(r[4 * i + 3]) * inv_l);
-          }
-        }
-        if (live)
-          p.part_lse[(static_cast<size_t>(split) * p.H + head) * p.T_q + row_g] =
-              l > 0.f ? (m2 + __log2f(l)) * 0.69314718056f : -INFINITY;
-      } else if (ok) {
-        tc_fence_after();
-        const float inv_l = 1.f / l;
-        const bool live = row_g < p.T_q;
-        __nv_bfloat16* const orow = p.out + (static_cast<size_t>(row_g) * p.H + head) * D;
-  #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + 32u * c, r);
-          tmem_wait_ld();
-          if (live) {
+          } else if (live) {
             uint32_t pk[16];
   #pragma unroll
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l,
                                   __uint_as_float(r[2 * i + 1]) * inv_l);
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D + 32 * c);
   #pragma unroll
             for (int i = 0; i < 4; ++i)
               dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
-        if (p.lse != nullptr && live)
-          p.lse[static_cast<size_t>(head) * p.T_q + row_g] = (m2 + __log2f(l)) * 0.69314718056f;
+        const float lse = l > 0.f ? (m2 + __log2f(l)) * 0.69314718056f : -INFINITY;
+        if (live && part)
+          p.part_lse[(static_cast<size_t>(split) * p.H + head) * p.T_q + row_g] = lse;
+        else if (live && p.lse != nullptr)
+          p.lse[static_cast<size_t>(head) * p.T_q + row_g] = lse;
       }
     }
   } else {
@@ -406,11 +404,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (b >= nb || t >= nk || tok >= n_max) return p.total_rows;
         return pool_row(p, pt_s, n_cached, tok);
       };
+      int ready = 0;                                        // chunks known to be published
       for (int j = 0; j < nk && ok; ++j) {
         const int coord = box_row(j, lane);                 // lane b resolves box b of tile j
         int cb[BN / 16];
   #pragma unroll
         for (int b = 0; b < BN / 16; ++b) cb[b] = __shfl_sync(0xffffffffu, coord, b);
+        if (kWaitPublished && lane == 0) {
+          // every chunk with a key in this tile must have been published
+          const int last_key = min((kb + j + 1) * BN, n_max) - 1;
+          const int ready0 = ready;
+          while (ok && ready < p.nchunks && (ready == 0 ? 0 : p.chunk_end[ready - 1]) <= last_key) {
+            ok = wait_flag(p.flags + ready, p.flag_gen, w);
+            ++ready;
+          }
+          if (ready != ready0) fence_proxy_async_global();
+        }
         if (lane == 0) {
   #pragma unroll
           for (int kv = 0; kv < 2 && ok; ++kv) {

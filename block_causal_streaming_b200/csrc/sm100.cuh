@@ -111,6 +111,40 @@ static __device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t par
   }
 }
 
+// System-scope acquire load of a flag written by another GPU (or the copy engine).
+__device__ __forceinline__ unsigned ld_acquire_sys(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Order this thread's earlier generic-proxy accesses to global memory (here: the acquire of a
+// publication flag) before its later async-proxy accesses (TMA loads of the published pages).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Wait until a publication flag reaches generation `gen` (compared as a signed 32-bit
+// difference, so generations may wrap).  Bounded exactly like mbar_wait.
+__device__ __forceinline__ bool wait_flag(const unsigned* flag, unsigned gen, const WaitCtx& w) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (static_cast<int>(ld_acquire_sys(flag) - gen) >= 0) return true;
+    if ((i & 15u) == 0) {
+      if (*w.cta_abort != 0) return false;
+      if (globaltimer_ns() - t0 > w.timeout_ns) {
+        raise_abort(w);
+        return false;
+      }
+      if (*reinterpret_cast<volatile unsigned*>(w.grid_abort) == w.launch_id) {
+        *w.cta_abort = 1;
+        return false;
+      }
+    }
+    __nanosleep(64);
+  }
+}
+
 // Wait for phase `parity` of `bar`.  Returns false (after raising the abort flags and recording
 // w.timeout_code) if the wait ran longer than w.timeout_ns, and false at once if another thread
 // of this CTA or another CTA of this launch already gave up.  Never spins without bound.

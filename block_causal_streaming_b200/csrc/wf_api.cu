@@ -16,6 +16,7 @@
 #include "attn_kernel.cuh"
 #include "attn_pair_kernel.cuh"
 #include "combine_kernel.cuh"
+#include "publish_kernel.cuh"
 
 // First error any kernel of this library recorded on this device (0 = none); cleared by
 // wf_check_status.
@@ -76,6 +77,12 @@ int device_state(DeviceState** out) {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  wfk::AttnSmem<128>::ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 wfk::AttnSmem<64>::ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<128, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 wfk::AttnSmem<128>::ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<64, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  wfk::AttnSmem<64>::ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(wfk::wf_attn_pair_kernel,
@@ -140,6 +147,25 @@ EncodeTiledFn encode_fn() {
                                          &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+typedef CUresult (*GetRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+// cuMemGetAddressRange from the driver, for the IPC helpers.
+GetRangeFn get_range_fn() {
+  static GetRangeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetRangeFn>(p);
     else
       cudaGetLastError();
   });
@@ -355,15 +381,19 @@ int launch_attention(AttnLaunch* L, cudaStream_t s) {
   p.launch_id = g_launch_counter.fetch_add(1);
   if (p.launch_id == 0) p.launch_id = g_launch_counter.fetch_add(1);
   const int64_t grid = static_cast<int64_t>(p.n_pairs) * p.H * p.n_splits;
+  const unsigned g = static_cast<unsigned>(grid);
+  const bool wait = p.flags != nullptr;
   if (L->use_pair)
-    wfk::wf_attn_pair_kernel<<<static_cast<unsigned>(2 * grid), wfk::kPairThreads,
-                               wfk::PairSmem::ALLOC, s>>>(p);
+    wfk::wf_attn_pair_kernel<<<2 * g, wfk::kPairThreads, wfk::PairSmem::ALLOC, s>>>(p);
+  else if (L->D == 128 && !wait)
+    wfk::wf_attn_fwd_kernel<128><<<g, wfk::kAttnThreads, wfk::AttnSmem<128>::ALLOC, s>>>(p);
   else if (L->D == 128)
-    wfk::wf_attn_fwd_kernel<128><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
-                                   wfk::AttnSmem<128>::ALLOC, s>>>(p);
+    wfk::wf_attn_fwd_kernel<128, true><<<g, wfk::kAttnThreads, wfk::AttnSmem<128>::ALLOC, s>>>(
+        p);
+  else if (!wait)
+    wfk::wf_attn_fwd_kernel<64><<<g, wfk::kAttnThreads, wfk::AttnSmem<64>::ALLOC, s>>>(p);
   else
-    wfk::wf_attn_fwd_kernel<64><<<static_cast<unsigned>(grid), wfk::kAttnThreads,
-                                  wfk::AttnSmem<64>::ALLOC, s>>>(p);
+    wfk::wf_attn_fwd_kernel<64, true><<<g, wfk::kAttnThreads, wfk::AttnSmem<64>::ALLOC, s>>>(p);
   if (cudaGetLastError() != cudaSuccess) return WF_ERR_CUDA;
   if (p.n_splits > 1) {
     const int64_t threads = static_cast<int64_t>(p.T_q) * p.H * 32;
@@ -510,6 +540,137 @@ int wf_attn_forward_split_noalloc(const void* q, const wf_kv_pool_t* kv_pages,
     set_split_buffers(&L, S, scratch);
   }
   return launch_attention(&L, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int wf_kv_append_publish(const wf_kv_pool_t* pool, uint32_t* flags, const wf_pool_dst_t* peers,
+                         int num_peers, int layer, int chunk, const void* k, const void* v,
+                         const int32_t* page_table, const wf_wavefront_t* wf, uint32_t generation,
+                         wf_stream_t stream) {
+  int rc = validate_pool(pool);
+  if (rc) return rc;
+  int t_kv = 0;
+  rc = validate_wavefront(wf, pool, &t_kv);
+  if (rc) return rc;
+  if (layer < 0 || chunk < 0 || chunk >= wf->num_chunks || page_table == nullptr ||
+      num_peers < 0 || num_peers > wfk::kMaxPublishDst - 1 || (num_peers > 0 && peers == nullptr))
+    return WF_ERR_INVALID_ARG;
+  for (int i = 0; i < num_peers; ++i)
+    if (peers[i].k_pool == nullptr || peers[i].v_pool == nullptr ||
+        !aligned16(peers[i].k_pool) || !aligned16(peers[i].v_pool) ||
+        (reinterpret_cast<uintptr_t>(peers[i].flags) & 3u))
+      return WF_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(flags) & 3u) return WF_ERR_INVALID_ARG;
+  const int t0 = wf->chunk_offsets[chunk];
+  const int rows = wf->chunk_offsets[chunk + 1] - t0;
+  if (rows > 0 && (k == nullptr || v == nullptr || !aligned16(k) || !aligned16(v)))
+    return WF_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  rc = device_state(&d);
+  if (rc) return rc;
+  wfk::PublishParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.k = static_cast<const uint4*>(k);
+  p.v = static_cast<const uint4*>(v);
+  p.pt_row = page_table + static_cast<int64_t>(layer) * wf->max_pages_per_seq;
+  p.status = d->status;
+  p.token0 = t0;
+  p.rows = rows;
+  p.vec_per_row = pool->num_heads * pool->head_dim * 2 / 16;
+  p.page_size = pool->page_size;
+  p.num_pages = pool->num_pages;
+  p.generation = generation;
+  const size_t flag_at = static_cast<size_t>(layer) * WF_MAX_CHUNKS + chunk;
+  p.n_dst = 1 + num_peers;
+  p.dst[0] = {static_cast<uint4*>(pool->k_pool), static_cast<uint4*>(pool->v_pool),
+              flags != nullptr ? flags + flag_at : nullptr};
+  for (int i = 0; i < num_peers; ++i)
+    p.dst[1 + i] = {static_cast<uint4*>(peers[i].k_pool), static_cast<uint4*>(peers[i].v_pool),
+                    peers[i].flags != nullptr ? peers[i].flags + flag_at : nullptr};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (rows > 0) {
+    const int warps_per_block = wfk::kPublishThreads / 32;
+    int blocks = (rows + warps_per_block - 1) / warps_per_block;
+    if (blocks > d->num_sms * 8) blocks = d->num_sms * 8;
+    wfk::wf_publish_kernel<<<blocks, wfk::kPublishThreads, 0, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return WF_ERR_CUDA;
+  }
+  wfk::wf_publish_flags_kernel<<<1, 32, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_attn_forward_published(const void* q, const wf_kv_pool_t* kv_pages,
+                              const int32_t* page_table_row, const wf_wavefront_t* wf,
+                              float scale, void* out, float* lse_or_null,
+                              const uint32_t* flags_row, uint32_t generation, int splits,
+                              void* workspace, size_t workspace_bytes, wf_stream_t stream) {
+  if (splits < 0 || flags_row == nullptr || (reinterpret_cast<uintptr_t>(flags_row) & 3u))
+    return WF_ERR_INVALID_ARG;
+  AttnLaunch L;
+  const int rc = prepare_attention(q, kv_pages, page_table_row, wf, scale, out, lse_or_null, &L);
+  if (rc || L.p.T_q == 0) return rc;
+  if (L.use_pair) return WF_ERR_SHAPE;         // the CTA-pair kernel has no publication wait
+  int S = splits > 0 ? splits : choose_splits(L.qp, L.p.H, L.d->num_sms);
+  S = std::min(S, max_splits(L.qp));
+  if (S > 1) {
+    const size_t need = split_workspace_bytes(L.qp, L.p.H, L.D, S);
+    if (workspace == nullptr || !aligned16(workspace)) return WF_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return WF_ERR_CAPACITY;
+    set_split_buffers(&L, S, workspace);
+  }
+  L.p.flags = flags_row;
+  L.p.flag_gen = generation;
+  L.p.nchunks = wf->num_chunks;
+  for (int c = 0; c < wf->num_chunks; ++c) L.p.chunk_end[c] = wf->chunk_offsets[c + 1];
+  return launch_attention(&L, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int wf_ipc_export(const void* device_ptr, void* handle64, size_t* offset) {
+  if (device_ptr == nullptr || handle64 == nullptr || offset == nullptr) return WF_ERR_INVALID_ARG;
+  // an IPC handle names a whole allocation: find its base (a pool may be a sub-range of a
+  // larger block of the caller's allocator) and report where device_ptr sits inside it
+  GetRangeFn range = get_range_fn();
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range == nullptr ||
+      range(&base, &size, reinterpret_cast<CUdeviceptr>(device_ptr)) != CUDA_SUCCESS)
+    return WF_ERR_CUDA;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) {
+    cudaGetLastError();
+    return WF_ERR_CUDA;
+  }
+  static_assert(sizeof(h) == 64, "CUDA IPC handles are 64 bytes");
+  std::memcpy(handle64, &h, sizeof(h));
+  *offset = static_cast<size_t>(reinterpret_cast<CUdeviceptr>(device_ptr) - base);
+  return WF_OK;
+}
+
+int wf_ipc_import(const void* handle64, size_t offset, void** device_ptr) {
+  if (handle64 == nullptr || device_ptr == nullptr) return WF_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle64, sizeof(h));
+  void* base = nullptr;
+  if (cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+    cudaGetLastError();
+    return WF_ERR_CUDA;
+  }
+  *device_ptr = static_cast<uint8_t*>(base) + offset;
+  return WF_OK;
+}
+
+int wf_ipc_close(void* device_ptr) {
+  if (device_ptr == nullptr) return WF_ERR_INVALID_ARG;
+  GetRangeFn range = get_range_fn();
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range == nullptr ||
+      range(&base, &size, reinterpret_cast<CUdeviceptr>(device_ptr)) != CUDA_SUCCESS)
+    return WF_ERR_CUDA;
+  if (cudaIpcCloseMemHandle(reinterpret_cast<void*>(base)) != cudaSuccess) {
+    cudaGetLastError();
+    return WF_ERR_CUDA;
+  }
+  return WF_OK;
 }
 
 int wf_selftest_timeout(unsigned timeout_us, wf_stream_t stream) {

@@ -177,6 +177,64 @@ int wf_attn_forward_split_noalloc(const void* q, const wf_kv_pool_t* kv_pages,
  */
 size_t wf_attn_workspace_size(const wf_wavefront_t* wf, int num_heads, int head_dim, int splits);
 
+/* ---------------------------------------------------------------------------------------------
+ * One-way K/V publication between GPUs (Wave Parallelism).  Every GPU owns one chunk of the
+ * wavefront and attends to the chunks before it; each producer writes its K/V, right after
+ * projection, straight into the attention buffers of every consumer, one way (project page, "03
+ * End-to-end KV transport", items 01-03; KipQuest "The deep dive").  Here all GPUs keep pools of
+ * the same geometry with the same page table, so a chunk lands in the same pages everywhere, and
+ * each pool has a flag array uint32 [num_layers][WF_MAX_CHUNKS] whose word (layer, chunk) holds
+ * the generation of the chunk's last publication.  Peer pools and flags are reached through
+ * pointers mapped with wf_ipc_import (or any other peer mapping); data moves by plain stores
+ * from this GPU's SMs over NVLink, never by TMA loads from a peer.
+ * --------------------------------------------------------------------------------------------- */
+typedef struct {
+  void* k_pool;        /* device bf16 pool of the destination GPU, same geometry as the source */
+  void* v_pool;
+  uint32_t* flags;     /* that GPU's flag array [num_layers][WF_MAX_CHUNKS], or NULL */
+} wf_pool_dst_t;
+
+/*
+ * wf_kv_append_publish -- wf_kv_append into `pool` and, in the same kernel, into every peer pool
+ * (up to 8), then a second kernel sets word (layer, chunk) of `flags` (this GPU's flag array, may
+ * be NULL) and of every peer's flags to `generation` with a system-scope release, after a
+ * system-wide fence.  Arguments as wf_kv_append plus `flags`, `peers[num_peers]` and
+ * `generation`.  An empty chunk only sets the flags.  Errors as wf_kv_append; WF_ERR_INVALID_ARG
+ * for more than 8 peers or a null/misaligned peer pool.  Asynchronous on `stream`.
+ */
+int wf_kv_append_publish(const wf_kv_pool_t* pool, uint32_t* flags, const wf_pool_dst_t* peers,
+                         int num_peers, int layer, int chunk, const void* k, const void* v,
+                         const int32_t* page_table, const wf_wavefront_t* wf, uint32_t generation,
+                         wf_stream_t stream);
+
+/*
+ * wf_attn_forward_published -- wf_attn_forward_split on chunks that other GPUs publish: before
+ * loading the keys of chunk c the kernel waits until flags_row[c] has reached `generation`
+ * (signed 32-bit difference >= 0, so generations may wrap), read with a system-scope acquire.
+ * flags_row: device uint32 [WF_MAX_CHUNKS], this layer's row of this GPU's flag array; every
+ * chunk the queries see (own chunk included) must be flagged, e.g. by wf_kv_append_publish.
+ * A wait that lasts longer than 2 s stops the kernel and records WF_ERR_TIMEOUT (read with
+ * wf_check_status).  Other arguments and errors as wf_attn_forward_split; WF_ERR_SHAPE if the
+ * library was built with the CTA-pair kernel.
+ */
+int wf_attn_forward_published(const void* q, const wf_kv_pool_t* kv_pages,
+                              const int32_t* page_table_row, const wf_wavefront_t* wf,
+                              float scale, void* out, float* lse_or_null,
+                              const uint32_t* flags_row, uint32_t generation, int splits,
+                              void* workspace, size_t workspace_bytes, wf_stream_t stream);
+
+/*
+ * wf_ipc_export / wf_ipc_import / wf_ipc_close -- share device memory (pools, flag arrays)
+ * between processes.  export writes the 64-byte IPC handle of the allocation containing
+ * device_ptr (cudaIpcGetMemHandle on its base) and device_ptr's byte offset inside it; import
+ * maps such a handle from another process with peer access enabled (cudaIpcOpenMemHandle) and
+ * returns base + offset; close unmaps the allocation containing an imported pointer.
+ * WF_ERR_CUDA on failure (e.g. a handle imported in the process that exported it).
+ */
+int wf_ipc_export(const void* device_ptr, void* handle64, size_t* offset);
+int wf_ipc_import(const void* handle64, size_t offset, void** device_ptr);
+int wf_ipc_close(void* device_ptr);
+
 /*
  * wf_check_status -- synchronise `stream`, then return and clear the first error any kernel of
  * this library recorded on the current device since the last call (WF_OK if none).  A pending

@@ -63,7 +63,7 @@ def _rank_main(rank, world, port, results):
 
 def test_replicas_take_the_slowest_rank_gloo():
     world = 2
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         results = m.dict()
         mp.start_processes(_rank_main, args=(world, _free_port(), results), nprocs=world,
                            start_method="spawn", join=True)
