@@ -10,8 +10,9 @@
 // One CTA = one unit of work: a head and 256 consecutive query rows (two 128-row Q tiles that
 // share every K/V tile they load).  Units are numbered so that the hardware's in-order block
 // dispatch runs the most expensive first (longest-processing-time order): kv_end is
-// non-decreasing in the query row, so blockIdx 0 takes the last 256 rows.  Heads vary fastest, so
-// the CTAs of all heads stream the same key range at about the same time and share it in L2.
+// non-decreasing in the query row, so blockIdx 0 takes the last 256 rows.  Heads vary fastest
+// (within groups of about 12 heads), so the CTAs of a group stream the same key range at about
+// the same time and share it in L2.
 //
 // Warp roles (384 threads):
 //   warps 0-3  softmax of Q tile 0: thread t owns query row t (TMEM lane t)
@@ -86,6 +87,7 @@ struct AttnParams {
   int* status;
   unsigned* grid_abort;
   int T_q, H, num_pages, page_size, total_rows, box_rows, n_pairs;
+  int head_group;     // heads per group of the dispatch order (divides H)
   int box_rows_v;     // V box rows (CTA-pair kernel: V half-tiles of 128 keys)
   float sl2;  // scale * log2(e)
   unsigned launch_id;
@@ -189,8 +191,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int unit = blockIdx.x / p.n_splits;
   const int split = blockIdx.x - unit * p.n_splits;
-  const int pair = p.n_pairs - 1 - unit / p.H;
-  const int head = unit % p.H;
+  // Heads are dispatched in groups of head_group: every row block of one group, longest first,
+  // heads fastest, before the next group -- so about as many CTAs read one head's keys at the
+  // same time as with 12 heads, whatever H is.
+  const int group_units = p.n_pairs * p.head_group;
+  const int group = unit / group_units, in_group = unit - group * group_units;
+  const int pair = p.n_pairs - 1 - in_group / p.head_group;
+  const int head = group * p.head_group + in_group % p.head_group;
   const int m0 = pair * (kNQT * kBM);
   const int last_row = min(m0 + kNQT * kBM, p.T_q) - 1;
   const int n_max = kv_end_of_row(p, last_row);        // keys any row of this unit may see

@@ -239,6 +239,15 @@ int unit_tiles(const QueryPlan& qp, int pair) {
   return (n + wfk::kBN - 1) / wfk::kBN;
 }
 
+// Heads per dispatch group: the fewest groups of at most kHeadsPerGroup heads that divide H
+// evenly (one group -- plain heads-fastest order -- when none does).
+constexpr int kHeadsPerGroup = 12;
+int head_group(int H) {
+  for (int g = (H + kHeadsPerGroup - 1) / kHeadsPerGroup; g <= H / 2; ++g)
+    if (H % g == 0 && H / g <= kHeadsPerGroup) return H / g;
+  return H;
+}
+
 // Every split must own at least one key tile of every unit.
 int max_splits(const QueryPlan& qp) {
   int m = kMaxSplits;
@@ -356,6 +365,7 @@ int prepare_attention(const void* q, const wf_kv_pool_t* kv_pages, const int32_t
   p.total_rows = static_cast<int>(total_rows);
   p.box_rows = box_rows;
   p.n_pairs = num_pairs(L->qp);
+  p.head_group = head_group(H);
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.nqc = L->qp.nqc;
   for (int c = 0; c < L->qp.nqc; ++c) {
