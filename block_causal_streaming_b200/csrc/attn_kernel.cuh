@@ -11,8 +11,8 @@
 // share every K/V tile they load).  Units are numbered so that the hardware's in-order block
 // dispatch runs the most expensive first (longest-processing-time order): kv_end is
 // non-decreasing in the query row, so blockIdx 0 takes the last 256 rows.  Heads vary fastest
-// (within groups of about 12 heads), so the CTAs of a group stream the same key range at about
-// the same time and share it in L2.
+// within groups of a few heads (the host picks the group size), so the CTAs of a group stream
+// the same key range at about the same time and share it in L2.
 //
 // Warp roles (384 threads):
 //   warps 0-3  softmax of Q tile 0: thread t owns query row t (TMEM lane t)
@@ -192,8 +192,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int unit = blockIdx.x / p.n_splits;
   const int split = blockIdx.x - unit * p.n_splits;
   // Heads are dispatched in groups of head_group: every row block of one group, longest first,
-  // heads fastest, before the next group -- so about as many CTAs read one head's keys at the
-  // same time as with 12 heads, whatever H is.
+  // heads fastest, before the next group -- so many CTAs read one head's keys at about the same
+  // time, whatever H is.
   const int group_units = p.n_pairs * p.head_group;
   const int group = unit / group_units, in_group = unit - group * group_units;
   const int pair = p.n_pairs - 1 - in_group / p.head_group;

@@ -240,8 +240,13 @@ int unit_tiles(const QueryPlan& qp, int pair) {
 }
 
 // Heads per dispatch group: the fewest groups of at most kHeadsPerGroup heads that divide H
-// evenly (one group -- plain heads-fastest order -- when none does).
-constexpr int kHeadsPerGroup = 12;
+// evenly (one group -- plain heads-fastest order -- when none does).  Measured on a B200 (p50,
+// 1.3B 5-step / 14B-shaped wavefronts): at most 1, 2, 3, 4, 6, 12 heads per group ->
+// 2.85 / 21.4, 2.84 / 18.3, 2.80 / 18.1, 2.79 / 18.3-18.5, 2.79 / 18.7, 2.85 / 19.3-19.7 ms.
+#ifndef WF_HEADS_PER_GROUP
+#define WF_HEADS_PER_GROUP 4
+#endif
+constexpr int kHeadsPerGroup = WF_HEADS_PER_GROUP;
 int head_group(int H) {
   for (int g = (H + kHeadsPerGroup - 1) / kHeadsPerGroup; g <= H / 2; ++g)
     if (H % g == 0 && H / g <= kHeadsPerGroup) return H / g;
