@@ -80,3 +80,15 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
 def test_arguments_are_checked():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])
+
+
+def test_workload_selection():
+    from block_causal_streaming_b200.workloads import WP_RANK0
+    assert bench.workload_of("2") is CONFIGS[2]
+    assert bench.workload_of("5") is CONFIGS[5]
+    assert bench.workload_of("wp") is WP_RANK0
+    with pytest.raises(SystemExit):
+        bench.main(["--config", "4"])          # the 30-layer round is a parity case, not a bench line
+    # one rank's call: one 4680-token chunk against 8 chunks of keys
+    assert (WP_RANK0.t_q, WP_RANK0.t_kv, WP_RANK0.num_ctx_chunks) == (4680, 37440, 7)
+    assert bench.attention_flops(WP_RANK0) == 4 * 128 * 12 * 4680 * 37440
