@@ -28,8 +28,9 @@
 //                         __syncwarp, so one cluster-scope arrive per warp, not per thread)
 //   x_max, x_sum          each CTA, count 256: the two softmax warpgroups swap row maxima / sums
 // Measured on the 1.3B 5-step wavefront this kernel is correct but slower than attn_kernel.cuh
-// (4.53 vs 3.4-3.6 ms): the cross-CTA hand-offs cost more than the tensor time they save.  It is
-// launched only when the library is compiled with WF_ATTN_PAIR=1.
+// (4.53 ms against 3.4-3.6 ms for the single-CTA kernel of the time, 2.8 ms now): the cross-CTA
+// hand-offs cost more than the tensor time they save.  It is launched only when the library is
+// compiled with WF_ATTN_PAIR=1.
 #pragma once
 
 #include <cuda_bf16.h>
