@@ -204,3 +204,20 @@ def test_bounded_wait_runs_out_and_context_survives():
     out = run(layer, q)
     assert check_status() == WF_OK
     assert_parity(out.float().cpu().numpy(), full_oracle(wl, inp, with_lse=False), "after timeout")
+
+
+def test_sixty_four_chunks_the_descriptor_maximum():
+    """WF_MAX_CHUNKS chunks: 4 context + 60 query chunks of 1..40 tokens, every element."""
+    import random
+    rnd = random.Random(64)
+    ctx = tuple(rnd.randint(5, 30) for _ in range(4))
+    act = tuple(rnd.randint(1, 40) for _ in range(60))
+    wl = small_case("sixty_four_chunks", 2, 128, ctx, act, 16, seed=64)
+    assert wl.num_chunks == 64
+    inp = make_inputs(wl)
+    layer, q, _, _ = place(wl, inp, fill=float("nan"))
+    out, lse = run(layer, q, with_lse=True)
+    assert check_status() == WF_OK
+    ref, ref_lse = full_oracle(wl, inp)
+    assert_parity(out.float().cpu().numpy(), ref, wl.name)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=2e-3)

@@ -146,3 +146,15 @@ def test_a_chunk_never_published_times_out_and_the_device_stays_usable():
     ref = oracle.attention(P.inp.q, P.inp.k, P.inp.v, CASE.chunk_offsets, CASE.num_ctx_chunks,
                            scale_of(CASE))
     assert_parity(out.float().cpu().numpy(), ref, "after a timeout")
+
+
+def test_publication_at_head_dim_64_with_splits():
+    wl = small_case("publish_d64", 3, 64, (100,), (90, 150), 16, seed=52)
+    P = Published(wl, n_peers=2)
+    P.publish(range(wl.num_chunks))
+    ref = oracle.attention(P.inp.q, P.inp.k, P.inp.v, wl.chunk_offsets, wl.num_ctx_chunks,
+                           scale_of(wl))
+    for i in (1, 2):
+        out = P.attend(i, splits=2)
+        assert check_status() == WF_OK
+        assert_parity(out.float().cpu().numpy(), ref, f"pool {i}")

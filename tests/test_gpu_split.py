@@ -98,3 +98,20 @@ def test_wave_parallel_rank_call_library_choice_sampled_parity():
     # the single pass agrees within the parity bar too
     single = run(layer, q)
     assert_parity(single[rows, heads].float().cpu().numpy(), ref, wl.name + " single pass")
+
+
+def test_sixteen_splits_the_maximum():
+    """A unit of 20 key tiles split 16 ways (and a request for more is capped at 16)."""
+    wl = small_case("split_16", 1, 128, (2300,), (200,), 64, seed=35)
+    inp = make_inputs(wl)
+    layer, q, _, _ = place(wl, inp)
+    assert attn_workspace_size(layer.desc, 1, 128, 40) == \
+        attn_workspace_size(layer.desc, 1, 128, 16)
+    ref, ref_lse = oracle_of(wl, inp)
+    for splits in (16, 40):
+        out = torch.empty_like(q)
+        lse = torch.empty(q.shape[1], q.shape[0], dtype=torch.float32, device=q.device)
+        layer.forward(q, out, lse=lse, splits=splits)
+        assert check_status() == WF_OK
+        assert_parity(out.float().cpu().numpy(), ref, f"S={splits}")
+        np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=2e-3)
