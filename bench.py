@@ -1,6 +1,6 @@
 """Benchmark: block-causal chunk attention over a Wan2.1-1.3B-shaped 5-step wavefront.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {wf,reference}] [--config 2]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {wf,reference}] [--workload W]
 
 One step is one pass of the whole hot path over one layer of the wavefront: wf_kv_append of the
 five active chunks' K/V into their pages (the two clean context chunks are appended once, before
@@ -13,9 +13,10 @@ Printed (rank 0, one JSON line): throughput in TFLOP/s of algorithmic attention 
 with tokens/s, the roofline of the attention kernel, an end-to-end figure through the C ABI with
 host buffers, the CPU oracle as a baseline, and the SM clocks seen during the timed region.
 
---config 3 / 5 run the other full-size wavefronts; --config wp runs one Wave-Parallelism rank's
-call (one 4680-token chunk against a 37 440-key prefix) through wf_attn_forward_split with the
-library's choice of key splits, whose timed attention then includes the merge kernel.
+--workload wan13b_4step / wan14b run the other full-size wavefronts; --workload wp_rank0 runs one
+Wave-Parallelism rank's call (one 4680-token chunk against a 37 440-key prefix) through
+wf_attn_forward_split with the library's choice of key splits, whose timed attention then
+includes the merge kernel.
 
 With --gpus N > 1 (launched by torch.distributed.run) every rank runs an independent replica of
 the same workload: the path has no exchange step, so there is no data-path collective; a barrier
@@ -39,7 +40,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from block_causal_streaming_b200.workloads import (CONFIGS, WP_RANK0, Workload,  # noqa: E402
+from block_causal_streaming_b200.workloads import (WORKLOADS, WP_RANK0, Workload,  # noqa: E402
                                                    make_inputs)
 
 METRIC = "block-causal chunk-attention TFLOP/s and % of B200 bf16 peak; tokens/s"
@@ -52,8 +53,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ------------------------------------------------------------------------------ accounting
-def workload_of(config: str) -> Workload:
-    return WP_RANK0 if config == "wp" else CONFIGS[int(config)]
+BENCH_WORKLOADS = ("wan13b_5step", "wan13b_4step", "wan14b", "wp_rank0")
+
+
+def workload_of(name: str) -> Workload:
+    return WORKLOADS[name]
 
 
 def attention_flops(wl: Workload) -> int:
@@ -248,7 +252,7 @@ def gpu_arm(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     init_dist(world, "nccl")
-    wl = workload_of(args.config)
+    wl = workload_of(args.workload)
     inp = make_inputs(wl)
     H, D = wl.heads, wl.head_dim
     off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
@@ -265,7 +269,7 @@ def gpu_arm(args, world, rank, local):
     active = list(range(nctx, wl.num_chunks))
     layer.append_range(k, v, range(nctx))            # clean context: published once
     stream = torch.cuda.current_stream(dev)
-    splits = 0 if args.config == "wp" else None       # library-chosen key splits
+    splits = 0 if wl is WP_RANK0 else None            # library-chosen key splits
     split_used = splits is not None and wf.attn_workspace_size(layer.desc, H, D, 0) > 0
     launches_per_step = len(active) + 1 + (1 if split_used else 0)
 
@@ -425,7 +429,7 @@ def reference_arm(args, world, rank):
     """The oracle as it stands, on the host cores, on bounded samples of the same workload."""
     if rank != 0:
         return None
-    wl = workload_of(args.config)
+    wl = workload_of(args.workload)
     inp = make_inputs(wl)
     per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
     for i in range(args.warmup):
@@ -461,7 +465,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["wf", "reference"], default="wf")
-    ap.add_argument("--config", default="2", choices=["2", "3", "5", "wp"])
+    ap.add_argument("--workload", default="wan13b_5step", choices=BENCH_WORKLOADS)
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -118,8 +118,6 @@ WAN14B = Workload("wan14b_6ctx+5x4680_h40_d128_ps128", heads=40, head_dim=128,
                   active_stages=(200, 400, 600, 800, 1000), page_size=128,
                   value_scale=0.5, seed=4, page_order="perm")
 
-CONFIGS = {1: TINY, 2: WAN13B_5STEP, 3: WAN13B_4STEP, 4: WAN13B_ROUND30, 5: WAN14B}
-
 # One Wave-Parallelism rank's call: the critical consumer's single query chunk against a context
 # of 7 earlier chunks (8 chunks visible; project page, "02 Interactive pipeline", "Inside one
 # diffusion tick").  Seed 5; otherwise the 1.3B shapes above.
@@ -127,6 +125,10 @@ WP_RANK0 = Workload("wp_rank0_7ctx+1x4680_h12_d128", heads=12, head_dim=128,
                     ctx_lens=(CHUNK_TOKENS,) * 7, active_lens=(CHUNK_TOKENS,),
                     active_stages=(1000,), page_size=64, value_scale=0.5, seed=5,
                     page_order="perm")
+
+# The workloads by short name (bench.py --workload).
+WORKLOADS = {"tiny": TINY, "wan13b_5step": WAN13B_5STEP, "wan13b_4step": WAN13B_4STEP,
+             "wan13b_round30": WAN13B_ROUND30, "wan14b": WAN14B, "wp_rank0": WP_RANK0}
 
 
 def small_case(name: str, heads: int, head_dim: int, ctx_lens, active_lens, page_size: int,

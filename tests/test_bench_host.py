@@ -10,7 +10,8 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 import bench
-from block_causal_streaming_b200.workloads import CONFIGS, small_case
+from block_causal_streaming_b200.workloads import (TINY, WAN13B_5STEP, WAN14B, WP_RANK0,
+                                                   small_case)
 
 
 def _visible_pairs(wl):
@@ -21,7 +22,7 @@ def _visible_pairs(wl):
     return int((ids[None, :] <= q_ids[:, None]).sum())
 
 
-@pytest.mark.parametrize("wl", [CONFIGS[1],
+@pytest.mark.parametrize("wl", [TINY,
                                 small_case("acct", 3, 128, (50, 7), (33, 0, 90), 16, seed=1),
                                 small_case("acct2", 2, 64, (), (300,), 64, seed=2)],
                          ids=lambda w: w.name)
@@ -31,12 +32,12 @@ def test_flop_accounting_counts_only_visible_pairs(wl):
 
 def test_flop_accounting_of_benchmark_workloads():
     # 4*D*H*sum(len_c * end_c): 5 chunks of 4680 after 2 context chunks, H=12, D=128
-    assert bench.attention_flops(CONFIGS[2]) == 4 * 128 * 12 * sum(
+    assert bench.attention_flops(WAN13B_5STEP) == 4 * 128 * 12 * sum(
         4680 * 4680 * (c + 1) for c in range(2, 7))
 
 
 def test_row_flops_matches_total():
-    wl = CONFIGS[1]
+    wl = TINY
     assert bench.rows_flops(wl, range(wl.t_q), wl.heads) == bench.attention_flops(wl)
 
 
@@ -83,12 +84,11 @@ def test_arguments_are_checked():
 
 
 def test_workload_selection():
-    from block_causal_streaming_b200.workloads import WP_RANK0
-    assert bench.workload_of("2") is CONFIGS[2]
-    assert bench.workload_of("5") is CONFIGS[5]
-    assert bench.workload_of("wp") is WP_RANK0
-    with pytest.raises(SystemExit):
-        bench.main(["--config", "4"])          # the 30-layer round is a parity case, not a bench line
+    assert bench.workload_of("wan13b_5step") is WAN13B_5STEP
+    assert bench.workload_of("wan14b") is WAN14B
+    assert bench.workload_of("wp_rank0") is WP_RANK0
+    with pytest.raises(SystemExit):            # the 30-layer round is a parity case, not a bench line
+        bench.main(["--workload", "wan13b_round30"])
     # one rank's call: one 4680-token chunk against 8 chunks of keys
     assert (WP_RANK0.t_q, WP_RANK0.t_kv, WP_RANK0.num_ctx_chunks) == (4680, 37440, 7)
     assert bench.attention_flops(WP_RANK0) == 4 * 128 * 12 * 4680 * 37440

@@ -6,7 +6,7 @@ import torch
 import oracle
 from block_causal_streaming_b200 import WF_ERR_PAGE_OOB, WF_OK, check_status
 from block_causal_streaming_b200.layer import PagedPool, WavefrontLayer
-from block_causal_streaming_b200.workloads import CONFIGS, make_inputs, small_case
+from block_causal_streaming_b200.workloads import TINY, make_inputs, small_case
 
 pytestmark = pytest.mark.gpu
 
@@ -18,7 +18,7 @@ def as_bits(t: torch.Tensor) -> np.ndarray:
 
 
 @pytest.mark.parametrize("wl", [
-    CONFIGS[1],
+    TINY,
     small_case("append_ps48_shared_pages", 3, 128, (37, 11), (100, 5, 64), 48, seed=31,
                pool_pages=40),
     small_case("append_ps256", 2, 64, (300,), (513,), 256, seed=32, pool_pages=9),

@@ -13,7 +13,9 @@ import torch
 
 import oracle
 from block_causal_streaming_b200 import WF_ERR_PAGE_OOB, WF_OK, check_status
-from block_causal_streaming_b200.workloads import (CONFIGS, LayerInputs, make_inputs, make_layers,
+from block_causal_streaming_b200.workloads import (TINY, WAN13B_4STEP, WAN13B_5STEP,
+                                                   WAN13B_ROUND30, WAN14B, LayerInputs,
+                                                   make_inputs, make_layers,
                                                    small_case)
 from gpu_util import assert_parity, place, run, sample_rows, scale_of
 
@@ -48,8 +50,8 @@ def test_small_parity_every_element(wl):
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=2e-3)
 
 
-def test_config1_tiny_every_element():
-    wl = CONFIGS[1]
+def test_tiny_wavefront_every_element():
+    wl = TINY
     inp = make_inputs(wl)
     layer, q, _, _ = place(wl, inp)
     out = run(layer, q)
@@ -57,9 +59,8 @@ def test_config1_tiny_every_element():
     assert_parity(out.float().cpu().numpy(), full_oracle(wl, inp, with_lse=False), wl.name)
 
 
-@pytest.mark.parametrize("cfg", [2, 3, 5])
-def test_full_size_config_sampled_parity(cfg):
-    wl = CONFIGS[cfg]
+@pytest.mark.parametrize("wl", [WAN13B_5STEP, WAN13B_4STEP, WAN14B], ids=lambda w: w.name)
+def test_full_size_wavefront_sampled_parity(wl):
     inp = make_inputs(wl)
     layer, q, _, _ = place(wl, inp, fill=float("nan"))
     out, lse = run(layer, q, with_lse=True)
@@ -67,7 +68,7 @@ def test_full_size_config_sampled_parity(cfg):
     assert check_status() == WF_OK
     assert torch.equal(out, out2), "two identical runs differ"
     assert torch.isfinite(out.float()).all()
-    rows, heads = sample_rows(wl, per_chunk=4, seed=cfg)
+    rows, heads = sample_rows(wl, per_chunk=4, seed=wl.seed)
     ref, ref_lse = oracle.attention_rows(inp.q, inp.k, inp.v, wl.chunk_offsets,
                                          wl.num_ctx_chunks, scale_of(wl), rows, heads,
                                          with_lse=True)
@@ -76,9 +77,9 @@ def test_full_size_config_sampled_parity(cfg):
     np.testing.assert_allclose(lse[heads, rows].cpu().numpy(), ref_lse, rtol=0, atol=2e-3)
 
 
-def test_config4_thirty_layer_round_sampled_parity():
+def test_thirty_layer_round_sampled_parity():
     """30 layers share one 4096-page pool; each layer appends its chunks, then attends."""
-    wl = CONFIGS[4]
+    wl = WAN13B_ROUND30
     layers = make_layers(wl)
     from block_causal_streaming_b200.layer import PagedPool, WavefrontLayer
     pool = PagedPool(wl.num_pages, wl.page_size, wl.heads, wl.head_dim, "cuda")
@@ -198,7 +199,7 @@ def test_bounded_wait_runs_out_and_context_survives():
     assert check_status() == WF_ERR_TIMEOUT
     assert time.perf_counter() - t0 < 5.0
     assert check_status() == WF_OK
-    wl = CONFIGS[1]
+    wl = TINY
     inp = make_inputs(wl)
     layer, q, _, _ = place(wl, inp)
     out = run(layer, q)
