@@ -97,7 +97,7 @@ def _ramp(n: int, lo: int, hi: int) -> tuple:
     return tuple(lo + (hi - lo) * i // (n - 1) for i in range(n))
 
 
-# The five workloads of the benchmark plan (index 1..5).
+# A tiny wavefront and synthetic wavefronts of the Wan2.1 1.3B and 14B shapes.
 TINY = Workload("tiny_3x48_h2_d64", heads=2, head_dim=64, ctx_lens=(),
                 active_lens=(48, 48, 48), active_stages=(200, 600, 1000), page_size=16,
                 value_scale=1.0, seed=0, page_order="identity")

@@ -1,6 +1,6 @@
 """wf_attn_forward on the GPU against the oracle.
 
-Parity bar (stated by the build's target): max-abs <= 1e-2 and mean-abs <= 1e-3 on bf16 outputs
+Parity bar: max-abs <= 1e-2 and mean-abs <= 1e-3 on bf16 outputs
 with fp32 accumulation.  Small cases are compared element by element on every output; the five
 benchmark workloads are compared on sampled rows (chunk edges, tile edges, the tail) plus
 properties that hold at any size.
