@@ -11,7 +11,8 @@ The product is the C-ABI library ``libwf_b200.so`` (declared in ``include/wf.h``
   (:mod:`.wave` maps the peers' pools between processes).
 
 This package is its thin Python binding (ctypes, argument marshalling only), a small helper that
-owns the paged pools of one layer (:mod:`.layer`) and the seeded synthetic workloads
+owns the paged pools of one layer (:mod:`.layer`), the round-by-round planner of a streaming
+window with an anchor and a rolling history (:mod:`.window`) and the seeded synthetic workloads
 (:mod:`.workloads`).  The binding is loaded on first use of any of its names and fails loudly if
 the library has not been built; there is no CPU fallback.
 """

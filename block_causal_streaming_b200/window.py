@@ -1,0 +1,212 @@
+"""Rolling context window for a streaming wavefront over one fixed paged layout.
+
+What a round contains (KipQuest summary of arXiv 2611.00859, "The deep dive"): chunks and
+denoising stages form a grid whose active cells lie on a diagonal that moves one chunk per round;
+the oldest active chunk is on its last stage and the newest has just left pure noise.  A chunk that
+has finished its last stage gets one more forward pass at the clean timestep, the *store* pass,
+whose keys and values become the history later chunks read.  Within a chunk attention is full;
+across chunks a chunk sees the anchor, the clean history, the live store and every earlier,
+cleaner chunk in flight, and never a later, noisier one.  The GitHub README ("Quick start",
+"Run the 4-step checkpoint") gives one store rank beside the denoising stages.  The project page
+("03 End-to-end KV transport", item 03 "Layout") has every producer write into its fixed slot of
+the consumer's attention buffer, with attention reading the prefix in place.
+
+Readings taken here, where the pages say no more:
+
+* The anchor is the first chunk ever stored.  It is kept for the whole stream.
+* The clean history holds the ``history`` most recently stored chunks after the anchor.  When a
+  newer one is stored, the oldest leaves.
+* Every chunk has the same number of tokens, ``chunk_len``: three latent frames in the Wan
+  configurations.
+
+Layout.  One layer's K/V occupy ``slots`` consecutive chunk slots of ``chunk_len`` tokens:
+
+    [anchor][history ring: ``history`` slots][live store][in flight, cleanest first]
+
+One page table per layer maps them, and it never changes.  Chunk slots are not page-aligned
+(4680 tokens is not a multiple of any page size the kernels take), so a slot's logical position
+cannot be moved by editing page-table entries.  Nothing that persists is moved, then:
+
+* The anchor and history chunks stay in their slots.  Every query sees all of them, and attention
+  over a set of keys does not depend on their order.  So the history is a ring: a newly stored chunk
+  takes the slot of the chunk it evicts.
+* The store chunk and the chunks in flight get new K/V every round.  They are appended each round
+  right after the last occupied history slot.
+* While the ring is filling, the store chunk already sits in the slot it keeps as history: nothing
+  is copied.  Once the ring is full, the store chunk sits past the ring.  After the round's
+  attention at a layer, its K/V are appended a second time, into the ring slot of the chunk that
+  leaves (``RoundView.store_to``).  That is one extra chunk append per layer per round.
+
+:class:`RollingWindow` is the host-side planner: a pure function from the round number to that
+round's descriptor.  :class:`RollingCache` holds the device pools and page tables.  Through the C
+ABI it runs one layer of a round: appends, attention and the hand-over into the ring.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import List, Optional, Sequence
+
+import torch
+
+ANCHOR, HISTORY, STORE, ACTIVE = "anchor", "history", "store", "active"
+MAX_CHUNKS = 64   # chunks per descriptor (WF_MAX_CHUNKS); the planner runs without the library
+
+
+@dataclasses.dataclass(frozen=True)
+class RoundView:
+    """One round's chunks in logical order (the order of the descriptor and of the slots)."""
+
+    round: int
+    chunk_ids: List[int]        # stream index of the chunk in each slot
+    roles: List[str]            # ANCHOR | HISTORY | STORE | ACTIVE per slot
+    chunk_stage: List[int]      # 0 for anchor, history and store; the timestep for chunks in flight
+    chunk_offsets: List[int]    # slot i holds logical tokens [i * chunk_len, (i + 1) * chunk_len)
+    num_ctx_chunks: int         # anchor + history: K/V only, no queries this round
+    store_to: Optional[int]     # slot that must also receive the store chunk's K/V after attention
+    evicted: Optional[int]      # stream index of the history chunk leaving after this round
+
+    @property
+    def num_chunks(self) -> int:
+        return len(self.chunk_ids)
+
+    @property
+    def query_slots(self) -> List[int]:
+        return list(range(self.num_ctx_chunks, self.num_chunks))
+
+    @property
+    def t_q(self) -> int:
+        return self.chunk_offsets[-1] - self.chunk_offsets[self.num_ctx_chunks]
+
+    def slot_of(self, chunk_id: int) -> int:
+        return self.chunk_ids.index(chunk_id)
+
+    def rank_view(self, slot: int) -> "RoundView":
+        """The call of the one rank whose query chunk is in ``slot`` (Wave Parallelism: one stage,
+        or the store pass, per GPU).  Its keys are the prefix up to and including that chunk, and
+        every earlier chunk is K/V only for it."""
+        if not self.num_ctx_chunks <= slot < self.num_chunks:
+            raise ValueError(f"slot {slot} carries no queries this round")
+        n = slot + 1
+        return dataclasses.replace(
+            self, chunk_ids=self.chunk_ids[:n], roles=self.roles[:n],
+            chunk_stage=self.chunk_stage[:n], chunk_offsets=self.chunk_offsets[:n + 1],
+            num_ctx_chunks=slot, store_to=None, evicted=None)
+
+
+class RollingWindow:
+    """Round-by-round plan of a streaming wavefront with a rolling history.
+
+    ``stages`` are the denoising timesteps of the in-flight positions, noisiest first (e.g.
+    1000, 800, 600, 400, 200).  Chunk ``c`` enters at round ``c``.  At round ``t`` it is on step
+    ``t - c``, and in the store pass at round ``c + len(stages)``.
+    """
+
+    def __init__(self, chunk_len: int, stages: Sequence[int], history: int, page_size: int):
+        stages = [int(s) for s in stages]
+        if chunk_len < 1 or history < 0 or not stages:
+            raise ValueError("chunk_len >= 1, history >= 0 and at least one stage are required")
+        if any(s <= 0 for s in stages) or any(a <= b for a, b in zip(stages, stages[1:])):
+            raise ValueError("stages must be positive and strictly decreasing (noisiest first)")
+        self.chunk_len = int(chunk_len)
+        self.stages = stages
+        self.history = int(history)
+        self.page_size = int(page_size)
+        self.slots = 1 + self.history + 1 + len(stages)
+        if self.slots > MAX_CHUNKS:
+            raise ValueError(f"{self.slots} chunk slots exceed the descriptor's {MAX_CHUNKS}")
+        self.tokens = self.slots * self.chunk_len
+        self.pages = math.ceil(self.tokens / self.page_size)
+
+    def ring_slot(self, chunk_id: int) -> int:
+        """Slot kept by a stored chunk: 0 for the anchor, then the ring."""
+        if chunk_id == 0:
+            return 0
+        if self.history == 0:
+            raise ValueError("no history is kept")
+        return 1 + (chunk_id - 1) % self.history
+
+    def view(self, t: int) -> RoundView:
+        if t < 0:
+            raise ValueError("rounds start at 0")
+        S, W, L = len(self.stages), self.history, self.chunk_len
+        last_stored = t - S - 1                      # chunks <= this finished their store pass
+        ids: List[int] = []
+        roles: List[str] = []
+        stage: List[int] = []
+        if last_stored >= 0:
+            ids.append(0)
+            roles.append(ANCHOR)
+            stage.append(0)
+            kept = list(range(max(1, last_stored - W + 1), last_stored + 1)) if W > 0 else []
+            by_slot = sorted(kept, key=self.ring_slot)
+            ids += by_slot
+            roles += [HISTORY] * len(by_slot)
+            stage += [0] * len(by_slot)
+        n_ctx = len(ids)
+        store = t - S
+        store_to = evicted = None
+        if store >= 0:
+            ids.append(store)
+            roles.append(STORE)
+            stage.append(0)
+            if store >= 1 and W > 0 and store - W >= 1:
+                # the ring is full: the store chunk takes the slot of the chunk that leaves
+                evicted = store - W
+                store_to = self.ring_slot(store)
+        for c in range(max(0, t - S + 1), t + 1):     # in flight, oldest (cleanest) first
+            ids.append(c)
+            roles.append(ACTIVE)
+            stage.append(self.stages[t - c])
+        offsets = [i * L for i in range(len(ids) + 1)]
+        return RoundView(round=t, chunk_ids=ids, roles=roles, chunk_stage=stage,
+                         chunk_offsets=offsets, num_ctx_chunks=n_ctx, store_to=store_to,
+                         evicted=evicted)
+
+
+class RollingCache:
+    """Device state of a rolling window: one K/V pool holding ``num_layers`` layers of
+    ``window.pages`` pages, and one fixed page-table row per layer.
+
+    Each round, for every layer: :meth:`run_layer` appends the round's query chunks (store pass
+    first, then the chunks in flight, in the order of :meth:`RollingWindow.view`).  It then runs
+    attention for all of them in one launch and, once the ring is full, hands the store chunk into
+    the slot of the chunk that leaves.
+    """
+
+    def __init__(self, window: RollingWindow, heads: int, head_dim: int, num_layers: int = 1,
+                 device="cuda", page_tables: Optional[torch.Tensor] = None,
+                 fill: Optional[float] = None):
+        from .layer import PagedPool
+        self.window = window
+        self.num_layers = int(num_layers)
+        self.pool = PagedPool(window.pages * self.num_layers, window.page_size, heads, head_dim,
+                              device, fill=fill)
+        if page_tables is None:
+            page_tables = torch.arange(window.pages * self.num_layers, dtype=torch.int32)
+            page_tables = page_tables.view(self.num_layers, window.pages)
+        if tuple(page_tables.shape) != (self.num_layers, window.pages):
+            raise ValueError("page_tables must be [num_layers, window.pages]")
+        self.page_tables = page_tables.to(device=device, dtype=torch.int32).contiguous()
+
+    def layer_view(self, view: RoundView, layer: int):
+        from .layer import WavefrontLayer
+        return WavefrontLayer(self.pool, self.page_tables, layer, view.chunk_offsets,
+                              view.chunk_stage, view.num_ctx_chunks)
+
+    def run_layer(self, view: RoundView, layer: int, q: torch.Tensor, k: torch.Tensor,
+                  v: torch.Tensor, out: torch.Tensor, scale: Optional[float] = None,
+                  lse: Optional[torch.Tensor] = None, stream=None) -> None:
+        """One layer of round ``view.round``.  ``q``, ``k``, ``v``, ``out``: bf16 [T_q, H, D], the
+        rows of the round's query chunks in logical order (store pass, then in flight)."""
+        if view.t_q == 0:
+            return
+        lay = self.layer_view(view, layer)
+        L = self.window.chunk_len
+        for i, slot in enumerate(view.query_slots):
+            lay.append(slot, k[i * L:(i + 1) * L], v[i * L:(i + 1) * L], stream)
+        lay.forward(q, out, scale=scale, lse=lse, stream=stream)
+        if view.store_to is not None:
+            # the store chunk is the first query chunk; after this layer's attention the evicted
+            # chunk is no longer read, so its slot takes the store chunk's clean K/V
+            lay.append(view.store_to, k[:L], v[:L], stream)

@@ -1,0 +1,144 @@
+"""The rolling-window planner (block_causal_streaming_b200.window) on the CPU.
+
+* Visible sets: for every round and every query chunk, the chunks its keys come from must be those
+  the pages name.  These are the anchor, the clean history, the live store and every earlier, cleaner
+  chunk in flight, and never a later, noisier one (KipQuest summary of arXiv 2611.00859, "The deep
+  dive").  The history is the ``history`` most recently stored chunks after the anchor.  The expected
+  set is written from the stream's chronology, not from the planner's slots.
+* Nothing that persists moves: a stored chunk keeps its logical token range from round to round.
+* Data flow: the appends the planner prescribes, replayed round after round with the oracle's
+  own paged scatter and gather, leave in every slot exactly the chunk the round's descriptor names,
+  bit for bit.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from block_causal_streaming_b200 import window as W
+
+SHAPES = [(1, 0), (1, 2), (2, 1), (4, 2), (5, 1), (5, 3), (3, 5)]   # (stages, history)
+
+
+def _stages(n):
+    return [1000 - i * (800 // max(n - 1, 1)) for i in range(n)] if n > 1 else [1000]
+
+
+def expected_visible(t, S, H, c, is_store):
+    """Stream indices visible to chunk ``c`` at round ``t``, from the chronology alone: chunk d
+    entered at round d, was in flight at rounds d..d+S-1, stored at round d+S."""
+    stored = [d for d in range(0, t - S)]                  # store pass finished before round t
+    history = [d for d in stored if d >= 1][-H:] if H > 0 else []
+    anchor = [0] if stored else []
+    if is_store:
+        return set(anchor) | set(history) | {c}
+    live_store = [t - S] if t - S >= 0 else []
+    in_flight_cleaner = [d for d in range(max(0, t - S + 1), t + 1) if d < c]
+    return set(anchor) | set(history) | set(live_store) | set(in_flight_cleaner) | {c}
+
+
+@pytest.mark.parametrize("S,H", SHAPES)
+def test_every_query_chunk_sees_exactly_what_the_pages_name(S, H):
+    win = W.RollingWindow(48, _stages(S), H, 16)
+    for t in range(0, 3 * (S + H) + 6):
+        v = win.view(t)
+        assert v.chunk_offsets == [i * 48 for i in range(v.num_chunks + 1)]
+        assert all(a <= b for a, b in zip(v.chunk_stage, v.chunk_stage[1:]))
+        assert v.num_chunks <= win.slots and v.chunk_offsets[-1] <= win.pages * 16
+        assert len(set(v.chunk_ids)) == v.num_chunks
+        for slot in v.query_slots:
+            c = v.chunk_ids[slot]
+            visible = set(v.chunk_ids[:slot + 1])       # the prefix rule of the descriptor
+            assert visible == expected_visible(t, S, H, c, v.roles[slot] == W.STORE), (t, c)
+            r = v.rank_view(slot)                        # the same set as one rank's own call
+            assert set(r.chunk_ids) == visible and r.num_ctx_chunks == slot
+            assert r.t_q == 48
+
+
+@pytest.mark.parametrize("S,H", SHAPES)
+def test_stored_chunks_never_move(S, H):
+    win = W.RollingWindow(40, _stages(S), H, 16)
+    prev = None
+    for t in range(0, 3 * (S + H) + 6):
+        v = win.view(t)
+        if prev is not None:
+            for slot in range(v.num_ctx_chunks):
+                c = v.chunk_ids[slot]
+                if prev.store_to is not None and c == prev.chunk_ids[prev.num_ctx_chunks]:
+                    assert slot == prev.store_to           # handed over into the evicted slot
+                elif c in prev.chunk_ids[:prev.num_ctx_chunks]:
+                    assert slot == prev.slot_of(c)         # stayed where it was
+                else:                                      # stored last round: no copy needed
+                    assert prev.roles[prev.slot_of(c)] == W.STORE and prev.slot_of(c) == slot
+                    assert prev.store_to is None
+        if v.evicted is not None:
+            assert v.store_to == v.slot_of(v.evicted)
+        prev = v
+
+
+@pytest.mark.parametrize("S,H,ps", [(2, 2, 16), (3, 1, 32), (1, 3, 16), (4, 0, 48)])
+def test_appends_replayed_with_the_oracle_leave_the_named_chunk_in_every_slot(S, H, ps):
+    """K/V content is a tag per (chunk, round, token); a stored chunk keeps its store-round tag."""
+    L, heads, D = 24, 1, 2                                   # 24 tokens: slots straddle pages
+    win = W.RollingWindow(L, _stages(S), H, ps)
+    rng = np.random.default_rng(3)
+    page_table = rng.permutation(win.pages)
+    pool = np.full((win.pages, ps, heads, D), -1, np.int64)
+    stored = {}                                              # chunk -> its store-round K rows
+
+    def rows(c, t):
+        base = (c * 1000 + t) * 100
+        return (base + np.arange(L * heads * D)).reshape(L, heads, D)
+
+    for t in range(0, 3 * (S + H) + 6):
+        v = win.view(t)
+        fresh = {v.chunk_ids[s]: rows(v.chunk_ids[s], t) for s in v.query_slots}
+        for s in v.query_slots:                              # the round's appends
+            oracle.scatter_chunk(pool, page_table, v.chunk_offsets[s], fresh[v.chunk_ids[s]])
+        logical = oracle.gather_logical(pool, page_table, v.chunk_offsets[-1])
+        for s, c in enumerate(v.chunk_ids):                  # what attention reads
+            want = fresh[c] if s >= v.num_ctx_chunks else stored[c]
+            got = logical[v.chunk_offsets[s]:v.chunk_offsets[s + 1]]
+            assert np.array_equal(got, want), (t, s, c)
+        if STORE_SLOT(v) is not None:
+            c = v.chunk_ids[STORE_SLOT(v)]
+            stored[c] = fresh[c]
+            if v.store_to is not None:                       # hand-over after attention
+                oracle.scatter_chunk(pool, page_table, v.chunk_offsets[v.store_to], fresh[c])
+                del stored[v.evicted]
+
+
+def STORE_SLOT(v):
+    return v.roles.index(W.STORE) if W.STORE in v.roles else None
+
+
+def test_pipeline_fill_and_steady_state_counts():
+    """4-step layout with two history chunks: the critical consumer (the noisiest chunk) sees
+    8 chunks in steady state, the cleanest chunk in flight 5 and the store pass 4 (project page,
+    "02 Interactive pipeline", "Inside one diffusion tick": r0 sees 8 chunks, r1-store about 5)."""
+    win = W.RollingWindow(4680, [1000, 750, 500, 250], 2, 64)
+    v = win.view(20)
+    assert v.roles == [W.ANCHOR, W.HISTORY, W.HISTORY, W.STORE] + [W.ACTIVE] * 4
+    assert [v.rank_view(s).num_chunks for s in v.query_slots] == [4, 5, 6, 7, 8]
+    assert v.chunk_stage == [0, 0, 0, 0, 250, 500, 750, 1000]
+    assert win.view(0).roles == [W.ACTIVE] and win.view(0).chunk_stage == [1000]
+    assert win.view(4).roles == [W.STORE] + [W.ACTIVE] * 4            # the anchor's store pass
+    assert win.slots == 8 and win.pages == 585
+
+
+def test_planner_argument_checks():
+    with pytest.raises(ValueError):
+        W.RollingWindow(48, [200, 1000], 1, 16)            # stages must decrease
+    with pytest.raises(ValueError):
+        W.RollingWindow(48, [1000], 63, 16)                # 65 slots > 64 chunks
+    with pytest.raises(ValueError):
+        W.RollingWindow(0, [1000], 1, 16)
+    v = W.RollingWindow(48, [1000, 500], 1, 16).view(5)
+    with pytest.raises(ValueError):
+        v.rank_view(0)                                     # the anchor carries no queries
+
+
+def test_max_chunks_matches_the_library():
+    from block_causal_streaming_b200 import build as wf_build
+    wf_build.build()
+    from block_causal_streaming_b200 import _abi
+    assert W.MAX_CHUNKS == _abi.WF_MAX_CHUNKS
