@@ -1,0 +1,98 @@
+"""Pins of the FP8 (e4m3) K/V oracle (oracle/fp8.py) against things other than itself.
+
+* The value table is checked against values the format's definition fixes one by one: the smallest
+  subnormal, the largest subnormal, the smallest normal, one, the largest finite value.  It must
+  also be strictly increasing.
+* The encoder is checked against PyTorch's own float8_e4m3fn cast, a library routine.  The sweep
+  covers every representable value, every midpoint between neighbours (the ties) and one ulp
+  either side of each midpoint, with both signs, up to 448.  PyTorch's cast does not saturate, so
+  above 448 the saturation reading is checked on its own.
+* Brute force: every code's value encodes back to that code.
+* Quantized rows: the largest element of a row maps to +-448 exactly.  A row of zeros gives scale 0.
+  Round trips stay within the format's error bound: half an ulp of a 3-bit mantissa, or half the
+  smallest subnormal, in units of the row scale.
+"""
+import numpy as np
+import torch
+
+from oracle import fp8
+
+
+def test_value_table_against_the_format_definition():
+    v = fp8.e4m3_values()
+    assert len(v) == 127 and np.all(np.diff(v) > 0)
+    assert v[0] == 0.0
+    assert v[0x01] == 2.0 ** -9                  # smallest subnormal: 1/8 * 2^(1-7)
+    assert v[0x07] == 7 * 2.0 ** -9              # largest subnormal
+    assert v[0x08] == 2.0 ** -6                  # smallest normal
+    assert v[0x38] == 1.0                        # exponent field 7 = bias
+    assert v[0x3C] == 1.5
+    assert v[0x7E] == 448.0 == fp8.E4M3_MAX      # 1.75 * 2^8
+    d = fp8.e4m3_decode(np.array([0x7F, 0xFF, 0x80, 0xB8, 0xFE], np.uint8))
+    assert np.isnan(d[0]) and np.isnan(d[1])
+    assert d[2] == 0.0 and np.signbit(d[2]) and d[3] == -1.0 and d[4] == -448.0
+
+
+def _sweep():
+    vals = fp8.e4m3_values().astype(np.float32)
+    mids = ((vals[:-1].astype(np.float64) + vals[1:]) / 2).astype(np.float32)
+    below = np.nextafter(mids, np.float32(0))
+    above = np.nextafter(mids, np.float32(1e9))
+    rng = np.random.default_rng(0)
+    rand = (rng.standard_normal(4000) * np.exp2(rng.integers(-12, 9, 4000))).astype(np.float32)
+    x = np.concatenate([vals, mids, below, above, rand])
+    x = x[np.abs(x) <= 448]
+    return np.concatenate([x, -x])
+
+
+def test_encoder_matches_pytorch_float8_e4m3fn_cast_in_range():
+    x = _sweep()
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = fp8.e4m3_encode(x)
+    assert np.array_equal(got, want)
+
+
+def test_every_code_round_trips_and_ties_go_to_the_even_code():
+    codes = np.arange(127, dtype=np.uint8)
+    vals = fp8.e4m3_decode(codes)
+    assert np.array_equal(fp8.e4m3_encode(vals), codes)
+    assert np.array_equal(fp8.e4m3_encode(-vals), codes | 0x80)
+    # midpoint of 1.0 (0x38) and 1.125 (0x39) -> 0x38; of 1.125 and 1.25 (0x3A) -> 0x3A
+    assert fp8.e4m3_encode(np.float32([1.0625, 1.1875])).tolist() == [0x38, 0x3A]
+    # half the smallest subnormal ties between 0 and 0x01 -> 0 (sign kept)
+    assert fp8.e4m3_encode(np.float32([2.0 ** -10, -2.0 ** -10])).tolist() == [0x00, 0x80]
+
+
+def test_saturation_above_the_largest_finite_value():
+    x = np.float32([448.0, 448.5, 463.9, 464.0, 479.0, 480.0, 1e6, 3e38])
+    assert fp8.e4m3_encode(x).tolist() == [0x7E] * len(x)
+    assert fp8.e4m3_encode(-x).tolist() == [0xFE] * len(x)
+
+
+def test_quantized_rows_hit_448_at_the_row_maximum_and_zero_rows_stay_zero():
+    rng = np.random.default_rng(1)
+    x = torch.from_numpy(rng.standard_normal((64, 3, 128)).astype(np.float32) *
+                         np.exp2(rng.integers(-20, 20, (64, 3, 1))).astype(np.float32))
+    x = x.bfloat16().float().numpy()
+    x[5, 1] = 0.0
+    codes, scale = fp8.quantize_rows(x)
+    assert codes.shape == x.shape and scale.shape == x.shape[:2]
+    idx = np.abs(x).argmax(axis=-1)
+    top = np.take_along_axis(codes, idx[..., None], -1)[..., 0]
+    live = scale > 0
+    assert np.all((top[live] & 0x7F) == 0x7E)
+    assert scale[5, 1] == 0 and not codes[5, 1].any()
+    back = fp8.dequantize_rows_f32(codes, scale).astype(np.float64)
+    err = np.abs(back - x)
+    bound = 2.0 ** -4 * np.abs(x) + 2.0 ** -10 * scale[..., None] * (1 + 1e-6) + 1e-30
+    assert np.all(err <= bound)
+
+
+def test_dequantized_rows_are_the_bf16_rounding_of_the_fp32_product():
+    codes = np.arange(256, dtype=np.uint8).reshape(2, 128)
+    codes[(codes & 0x7F) == 0x7F] = 0              # no NaN codes
+    scale = np.float32([0.37, 3.0e-3])
+    got = fp8.dequantize_rows(codes, scale).float().numpy()
+    prod = fp8.e4m3_decode(codes).astype(np.float64) * scale.astype(np.float64)[:, None]
+    # nearest bf16 of the product: within half a bf16 ulp (8 significand bits: 2^-8 relative)
+    assert np.all(np.abs(got - prod) <= np.abs(prod) * 2.0 ** -8 + 1e-38)
