@@ -245,6 +245,61 @@ def oracle_sample(wl: Workload, inp, target_s: float, seed: int = 0):
 
 
 # ------------------------------------------------------------------------------ GPU arm
+def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
+               hbm_peak: float) -> dict:
+    """The FP8 transport kernels over every chunk of the workload's layer: wf_kv_append_fp8
+    (bf16 rows -> e4m3 pages + per-(token, head) scales) and wf_kv_dequant (back into the bf16
+    pool), each leg timed with CUDA events on the launching stream after a 256 MB write that
+    flushes L2.  Algorithmic bytes: every K/V element read once and written once."""
+    import block_causal_streaming_b200 as wf
+    from block_causal_streaming_b200.layer import PagedPoolFp8
+    H, D, off = wl.heads, wl.head_dim, wl.chunk_offsets
+    fp = PagedPoolFp8(wl.num_pages, wl.page_size, H, D, dev)
+    flush = torch.empty(64 * 2 ** 20, dtype=torch.float32, device=dev)      # 256 MB > L2
+    chunks = range(wl.num_chunks)
+
+    def quant():
+        for c in chunks:
+            wf.kv_append_fp8(*fp.tensors, 0, c, k[off[c]:off[c + 1]], v[off[c]:off[c + 1]],
+                             layer.page_tables, layer.desc, stream)
+
+    def dequant():
+        for c in chunks:
+            wf.kv_dequant(*fp.tensors, layer.pool.k, layer.pool.v, 0, c, layer.page_tables,
+                          layer.desc, stream)
+
+    for _ in range(warmup):
+        quant()
+        dequant()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for e in evs:
+        flush.zero_()
+        e[0].record(stream)
+        quant()
+        e[1].record(stream)
+        flush.zero_()
+        e[2].record(stream)
+        dequant()
+        e[3].record(stream)
+    torch.cuda.synchronize(dev)
+    rc = wf.check_status()
+    if rc != wf.WF_OK:
+        raise RuntimeError(f"device status after the FP8 leg: {wf.strerror(rc)}")
+    rows = off[-1]
+    elems = 2 * rows * H * D                      # K and V
+    bf16_bytes, fp8_bytes = 2 * elems, elems + 2 * rows * H * 4
+    out = {"chunks": wl.num_chunks, "tokens": rows, "steps": steps,
+           "bytes_bf16": bf16_bytes, "bytes_fp8": fp8_bytes,
+           "bytes_ratio": round(fp8_bytes / bf16_bytes, 4), "peak_gbs": hbm_peak}
+    for name, (a, b) in (("append_fp8", (0, 1)), ("dequant", (2, 3))):
+        ms = statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
+        gbs = (bf16_bytes + fp8_bytes) / (ms / 1e3) / 1e9
+        out[name] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4),
+                     "launches": wl.num_chunks}
+    return out
+
+
 def gpu_arm(args, world, rank, local):
     import block_causal_streaming_b200 as wf
     from block_causal_streaming_b200.layer import PagedPool, WavefrontLayer
@@ -412,6 +467,9 @@ def gpu_arm(args, world, rank, local):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
     }
+    if args.fp8_kv:
+        res["fp8_kv"] = fp8_kv_leg(wl, layer, k, v, dev, stream, max(5, min(args.steps, 20)),
+                                   args.warmup, float(peaks["hbm_gbs"]))
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         tflops, info = oracle_sample(wl, inp, target_s=args.cpu_seconds)
         res["cpu_baseline"] = {"value": round(tflops, 6), "unit": UNIT,
@@ -469,6 +527,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8-kv", action="store_true",
+                    help="also time the FP8 K/V transport kernels (append to e4m3 pages, "
+                         "dequantize) on the workload's chunks")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -8,7 +8,9 @@ The product is the C-ABI library ``libwf_b200.so`` (declared in ``include/wf.h``
   for wavefronts with few query rows (one Wave-Parallelism rank's chunk against its prefix);
 * ``wf_kv_append_publish`` / ``wf_attn_forward_published`` -- one-way publication of a chunk's
   K/V into other GPUs' pools with a generation flag, and attention that waits for the flags
-  (:mod:`.wave` maps the peers' pools between processes).
+  (:mod:`.wave` maps the peers' pools between processes);
+* ``wf_kv_append_fp8`` / ``wf_kv_dequant`` -- a chunk's K/V as e4m3 codes with per-(token, head)
+  scales (half the bytes to move), and their conversion back into the bf16 pool.
 
 This package is its thin Python binding (ctypes, argument marshalling only), a small helper that
 owns the paged pools of one layer (:mod:`.layer`), the round-by-round planner of a streaming
@@ -22,7 +24,7 @@ _ABI_NAMES = (
     "WavefrontDesc", "WfError", "attn_forward", "check_status", "kv_append", "strerror",
     "selftest_timeout", "attn_forward_split", "attn_workspace_size",
     "attn_forward_split_noalloc", "kv_append_publish", "attn_forward_published", "ipc_export",
-    "ipc_import", "ipc_close", "PoolDst",
+    "ipc_import", "ipc_close", "PoolDst", "kv_append_fp8", "kv_dequant", "KvPoolFp8",
 )
 __all__ = list(_ABI_NAMES)
 

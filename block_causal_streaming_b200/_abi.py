@@ -28,7 +28,8 @@ WF_MAX_CHUNKS = 64
 EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror", "wf_version",
             "wf_selftest_timeout", "wf_attn_forward_split", "wf_attn_workspace_size",
             "wf_attn_forward_split_noalloc", "wf_kv_append_publish", "wf_attn_forward_published",
-            "wf_ipc_export", "wf_ipc_import", "wf_ipc_close")
+            "wf_ipc_export", "wf_ipc_import", "wf_ipc_close", "wf_kv_append_fp8",
+            "wf_kv_dequant")
 
 
 class WfError(RuntimeError):
@@ -45,6 +46,14 @@ class PoolDst(ctypes.Structure):
 
 class KvPool(ctypes.Structure):
     _fields_ = [("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p),
+                ("num_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+class KvPoolFp8(ctypes.Structure):
+    """wf_kv_pool_fp8_t: e4m3 codes [pages, page_size, H, D] and fp32 scales [pages, page_size, H]."""
+    _fields_ = [("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
+                ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
                 ("num_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
                 ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
 
@@ -106,6 +115,12 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wf_ipc_close.restype = i32
     lib.wf_attn_workspace_size.argtypes = [ctypes.POINTER(Wavefront), i32, i32, i32]
     lib.wf_attn_workspace_size.restype = ctypes.c_size_t
+    lib.wf_kv_append_fp8.argtypes = [ctypes.POINTER(KvPoolFp8), i32, i32, vp, vp,
+                                     ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(Wavefront), vp]
+    lib.wf_kv_append_fp8.restype = i32
+    lib.wf_kv_dequant.argtypes = [ctypes.POINTER(KvPoolFp8), ctypes.POINTER(KvPool), i32, i32,
+                                  ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(Wavefront), vp]
+    lib.wf_kv_dequant.restype = i32
     return lib
 
 
@@ -147,6 +162,7 @@ def _stream_handle(stream) -> Optional[int]:
 def _check_tensor(t, name: str, dtype_name: str):
     import torch
     want = {"bf16": (torch.bfloat16,), "i32": (torch.int32,), "f32": (torch.float32,),
+            "u8": (torch.uint8,),
             "u32": (torch.int32, torch.uint32)}[dtype_name]      # flag words: any 32-bit int
     if t.dtype not in want:
         raise TypeError(f"{name}: expected {want[0]}, got {t.dtype}")
@@ -170,6 +186,50 @@ def kv_append(k_pool, v_pool, layer: int, chunk: int, k, v, page_table, wf: Wave
                           ctypes.byref(wf.c), _stream_handle(stream))
     if rc != WF_OK:
         raise WfError(rc, "wf_kv_append")
+
+
+def _fp8_pool_struct(k_codes, v_codes, k_scale, v_scale) -> KvPoolFp8:
+    num_pages, page_size, H, D = (int(x) for x in k_codes.shape)
+    for t, n, d in ((k_codes, "k_codes", "u8"), (v_codes, "v_codes", "u8"),
+                    (k_scale, "k_scale", "f32"), (v_scale, "v_scale", "f32")):
+        _check_tensor(t, n, d)
+    if tuple(v_codes.shape) != tuple(k_codes.shape) or \
+            tuple(k_scale.shape) != (num_pages, page_size, H) or \
+            tuple(v_scale.shape) != (num_pages, page_size, H):
+        raise ValueError("FP8 pool: codes [pages, page_size, H, D] and scales [pages, page_size, H]")
+    return KvPoolFp8(k_codes.data_ptr(), v_codes.data_ptr(), k_scale.data_ptr(),
+                     v_scale.data_ptr(), num_pages, page_size, H, D)
+
+
+def kv_append_fp8(k_codes, v_codes, k_scale, v_scale, layer: int, chunk: int, k, v, page_table,
+                  wf: WavefrontDesc, stream=None) -> None:
+    """wf_kv_append_fp8: quantize chunk ``chunk``'s K/V ([L, H, D] bf16) to e4m3 codes with one
+    fp32 scale per (token, head) row, into an FP8 pool through row ``layer`` of ``page_table``."""
+    for t, n, d in ((k, "k", "bf16"), (v, "v", "bf16"), (page_table, "page_table", "i32")):
+        _check_tensor(t, n, d)
+    pool = _fp8_pool_struct(k_codes, v_codes, k_scale, v_scale)
+    rc = lib.wf_kv_append_fp8(ctypes.byref(pool), int(layer), int(chunk), k.data_ptr(),
+                              v.data_ptr(), ctypes.cast(ctypes.c_void_p(page_table.data_ptr()),
+                                                        ctypes.POINTER(ctypes.c_int32)),
+                              ctypes.byref(wf.c), _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_kv_append_fp8")
+
+
+def kv_dequant(k_codes, v_codes, k_scale, v_scale, k_pool, v_pool, layer: int, chunk: int,
+               page_table, wf: WavefrontDesc, stream=None) -> None:
+    """wf_kv_dequant: chunk ``chunk`` of an FP8 pool -> the same rows of a bf16 pool."""
+    for t, n, d in ((k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
+                    (page_table, "page_table", "i32")):
+        _check_tensor(t, n, d)
+    src = _fp8_pool_struct(k_codes, v_codes, k_scale, v_scale)
+    dst = _pool_struct(k_pool, v_pool)
+    rc = lib.wf_kv_dequant(ctypes.byref(src), ctypes.byref(dst), int(layer), int(chunk),
+                           ctypes.cast(ctypes.c_void_p(page_table.data_ptr()),
+                                       ctypes.POINTER(ctypes.c_int32)),
+                           ctypes.byref(wf.c), _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_kv_dequant")
 
 
 def attn_forward(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: float, out,

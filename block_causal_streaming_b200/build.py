@@ -20,6 +20,7 @@ SOURCES = [os.path.join(CSRC, "wf_api.cu")]
 DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "attn_kernel.cuh",
                                                       "attn_pair_kernel.cuh",
                                                       "append_kernel.cuh", "combine_kernel.cuh",
+                                                      "fp8_kernel.cuh",
                                                       "publish_kernel.cuh")] + \
     [os.path.join(ROOT, "include", "wf.h")]
 

@@ -16,6 +16,7 @@
 #include "attn_kernel.cuh"
 #include "attn_pair_kernel.cuh"
 #include "combine_kernel.cuh"
+#include "fp8_kernel.cuh"
 #include "publish_kernel.cuh"
 
 // First error any kernel of this library recorded on this device (0 = none); cleared by
@@ -686,6 +687,111 @@ int wf_ipc_close(void* device_ptr) {
     return WF_ERR_CUDA;
   }
   return WF_OK;
+}
+
+namespace {
+
+int validate_pool_fp8(const wf_kv_pool_fp8_t* pool) {
+  if (pool == nullptr || pool->k_codes == nullptr || pool->v_codes == nullptr ||
+      pool->k_scale == nullptr || pool->v_scale == nullptr)
+    return WF_ERR_INVALID_ARG;
+  if (!aligned16(pool->k_codes) || !aligned16(pool->v_codes) || !aligned16(pool->k_scale) ||
+      !aligned16(pool->v_scale))
+    return WF_ERR_INVALID_ARG;
+  // the same geometry rules as a bf16 pool
+  wf_kv_pool_t g{pool->k_codes, pool->v_codes, pool->num_pages, pool->page_size, pool->num_heads,
+                 pool->head_dim};
+  return validate_pool(&g);
+}
+
+// Checks shared by the FP8 calls; on success *t0 / *rows are the chunk's token range and *row its
+// page-table row.
+int fp8_chunk_args(const wf_kv_pool_fp8_t* pool, int layer, int chunk, const int32_t* page_table,
+                   const wf_wavefront_t* wf, int* t0, int* rows, const int32_t** row) {
+  int rc = validate_pool_fp8(pool);
+  if (rc) return rc;
+  wf_kv_pool_t g{pool->k_codes, pool->v_codes, pool->num_pages, pool->page_size, pool->num_heads,
+                 pool->head_dim};
+  int t_kv = 0;
+  rc = validate_wavefront(wf, &g, &t_kv);
+  if (rc) return rc;
+  if (layer < 0 || chunk < 0 || chunk >= wf->num_chunks || page_table == nullptr)
+    return WF_ERR_INVALID_ARG;
+  *t0 = wf->chunk_offsets[chunk];
+  *rows = wf->chunk_offsets[chunk + 1] - *t0;
+  *row = page_table + static_cast<int64_t>(layer) * wf->max_pages_per_seq;
+  return WF_OK;
+}
+
+int fp8_blocks(const DeviceState* d, int rows, int heads) {
+  const int64_t warps = static_cast<int64_t>(rows) * heads;
+  const int per_block = wfk::kFp8Threads / 32;
+  int64_t blocks = (warps + per_block - 1) / per_block;
+  const int64_t cap = static_cast<int64_t>(d->num_sms) * 8;   // 64 warps per SM in flight
+  return static_cast<int>(blocks < cap ? blocks : cap);
+}
+
+}  // namespace
+
+int wf_kv_append_fp8(const wf_kv_pool_fp8_t* pool, int layer, int chunk, const void* k,
+                     const void* v, const int32_t* page_table, const wf_wavefront_t* wf,
+                     wf_stream_t stream) {
+  int t0 = 0, rows = 0;
+  const int32_t* row = nullptr;
+  int rc = fp8_chunk_args(pool, layer, chunk, page_table, wf, &t0, &rows, &row);
+  if (rc) return rc;
+  if (rows == 0) return WF_OK;
+  if (k == nullptr || v == nullptr || !aligned16(k) || !aligned16(v)) return WF_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  rc = device_state(&d);
+  if (rc) return rc;
+  const int blocks = fp8_blocks(d, rows, pool->num_heads);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto ks = static_cast<const __nv_bfloat16*>(k);
+  auto vs = static_cast<const __nv_bfloat16*>(v);
+  auto kc = static_cast<uint8_t*>(pool->k_codes);
+  auto vc = static_cast<uint8_t*>(pool->v_codes);
+  if (pool->head_dim == 128)
+    wfk::wf_quant_append_kernel<128><<<blocks, wfk::kFp8Threads, 0, s>>>(
+        ks, vs, kc, vc, pool->k_scale, pool->v_scale, row, t0, rows, pool->num_heads,
+        pool->page_size, pool->num_pages, d->status);
+  else
+    wfk::wf_quant_append_kernel<64><<<blocks, wfk::kFp8Threads, 0, s>>>(
+        ks, vs, kc, vc, pool->k_scale, pool->v_scale, row, t0, rows, pool->num_heads,
+        pool->page_size, pool->num_pages, d->status);
+  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_kv_dequant(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int layer, int chunk,
+                  const int32_t* page_table, const wf_wavefront_t* wf, wf_stream_t stream) {
+  int t0 = 0, rows = 0;
+  const int32_t* row = nullptr;
+  int rc = fp8_chunk_args(src, layer, chunk, page_table, wf, &t0, &rows, &row);
+  if (rc) return rc;
+  rc = validate_pool(dst);
+  if (rc) return rc;
+  if (dst->num_pages != src->num_pages || dst->page_size != src->page_size ||
+      dst->num_heads != src->num_heads || dst->head_dim != src->head_dim)
+    return WF_ERR_SHAPE;
+  if (rows == 0) return WF_OK;
+  DeviceState* d = nullptr;
+  rc = device_state(&d);
+  if (rc) return rc;
+  const int blocks = fp8_blocks(d, rows, src->num_heads);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto kc = static_cast<const uint8_t*>(src->k_codes);
+  auto vc = static_cast<const uint8_t*>(src->v_codes);
+  auto kp = static_cast<__nv_bfloat16*>(dst->k_pool);
+  auto vp = static_cast<__nv_bfloat16*>(dst->v_pool);
+  if (src->head_dim == 128)
+    wfk::wf_dequant_kernel<128><<<blocks, wfk::kFp8Threads, 0, s>>>(
+        kc, vc, src->k_scale, src->v_scale, kp, vp, row, t0, rows, src->num_heads,
+        src->page_size, src->num_pages, d->status);
+  else
+    wfk::wf_dequant_kernel<64><<<blocks, wfk::kFp8Threads, 0, s>>>(
+        kc, vc, src->k_scale, src->v_scale, kp, vp, row, t0, rows, src->num_heads,
+        src->page_size, src->num_pages, d->status);
+  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
 int wf_selftest_timeout(unsigned timeout_us, wf_stream_t stream) {

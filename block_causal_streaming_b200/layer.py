@@ -28,6 +28,25 @@ class PagedPool:
         self.num_pages, self.page_size, self.heads, self.head_dim = shape
 
 
+class PagedPoolFp8:
+    """FP8 K/V pool with the geometry of a :class:`PagedPool`: e4m3 codes uint8
+    [num_pages, page_size, H, D] and one fp32 scale per (token, head) row [num_pages, page_size, H]
+    for K and for V.  Filled by wf_kv_append_fp8, read back by wf_kv_dequant."""
+
+    def __init__(self, num_pages: int, page_size: int, heads: int, head_dim: int,
+                 device="cuda"):
+        shape = (num_pages, page_size, heads, head_dim)
+        self.k_codes = torch.zeros(shape, dtype=torch.uint8, device=device)
+        self.v_codes = torch.zeros(shape, dtype=torch.uint8, device=device)
+        self.k_scale = torch.zeros(shape[:3], dtype=torch.float32, device=device)
+        self.v_scale = torch.zeros(shape[:3], dtype=torch.float32, device=device)
+        self.num_pages, self.page_size, self.heads, self.head_dim = shape
+
+    @property
+    def tensors(self):
+        return self.k_codes, self.v_codes, self.k_scale, self.v_scale
+
+
 class WavefrontLayer:
     """One layer of a wavefront: its descriptor and its page-table rows.
 

@@ -236,6 +236,47 @@ int wf_ipc_import(const void* handle64, size_t offset, void** device_ptr);
 int wf_ipc_close(void* device_ptr);
 
 /*
+ * FP8 K/V pages for transport (project page, "03 End-to-end KV transport", item 01 "Precision":
+ * K/V sent in FP8 halve the bytes the producers move and are converted back before attention).
+ * An FP8 pool has the geometry of a bf16 pool and is addressed through the same page table:
+ * e4m3 codes (sign, 4 exponent bits with bias 7, 3 mantissa bits; no infinities; largest finite
+ * magnitude 448) in [num_pages][page_size][num_heads][head_dim] bytes, and one fp32 scale per
+ * (token, head) row in [num_pages][page_size][num_heads].  A per-page scale is not used: two
+ * chunks may share a page.  All four pointers are device memory owned by the caller, 16-byte
+ * aligned.
+ */
+typedef struct {
+  void* k_codes;
+  void* v_codes;
+  float* k_scale;
+  float* v_scale;
+  int32_t num_pages;
+  int32_t page_size;   /* tokens per page: a positive multiple of 16 */
+  int32_t num_heads;
+  int32_t head_dim;    /* 64 or 128 */
+} wf_kv_pool_fp8_t;
+
+/*
+ * wf_kv_append_fp8 -- wf_kv_append into an FP8 pool.  Each (token, head) row x of head_dim values,
+ * with amax its largest magnitude, is stored as scale = amax / 448 and codes
+ * e4m3(x * (448 / amax)), rounded to nearest even and saturated at +-448; both divisions and
+ * the product are fp32 round-to-nearest.  A row of zeros stores scale 0 and zero codes.
+ * Arguments and errors as wf_kv_append (k, v: device bf16 [L_c][H][D], 16-byte aligned).
+ */
+int wf_kv_append_fp8(const wf_kv_pool_fp8_t* pool, int layer, int chunk, const void* k,
+                     const void* v, const int32_t* page_table, const wf_wavefront_t* wf,
+                     wf_stream_t stream);
+
+/*
+ * wf_kv_dequant -- write chunk `chunk` of layer `layer` from the FP8 pool `src` into the bf16 pool
+ * `dst` (same geometry, same page table): value = bf16_rne(decode(code) * scale).  Only that
+ * chunk's rows of `dst` are written.  Errors as wf_kv_append; WF_ERR_SHAPE if the two pools'
+ * geometries differ.  Attention then reads `dst` as usual.
+ */
+int wf_kv_dequant(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int layer, int chunk,
+                  const int32_t* page_table, const wf_wavefront_t* wf, wf_stream_t stream);
+
+/*
  * wf_check_status -- synchronise `stream`, then return and clear the first error any kernel of
  * this library recorded on the current device since the last call (WF_OK if none).  A pending
  * CUDA error on the stream is returned as WF_ERR_CUDA.

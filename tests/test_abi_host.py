@@ -158,3 +158,40 @@ def test_split_validation_errors_without_a_gpu(abi):
         abi.WF_ERR_STAGE_ORDER
     empty = abi.WavefrontDesc([0, 64, 64], [0, 0], 1, 8)
     assert split(_pool(abi), empty) == abi.WF_OK
+
+
+def _fp8_pool(abi, **kw):
+    args = dict(k_codes=FAKE, v_codes=FAKE, k_scale=FAKE, v_scale=FAKE, num_pages=8, page_size=64,
+                num_heads=2, head_dim=128)
+    args.update(kw)
+    return abi.KvPoolFp8(**args)
+
+
+def test_fp8_validation_errors_without_a_gpu(abi):
+    desc = abi.WavefrontDesc([0, 64, 128, 200], [0, 200, 1000], 1, 8)
+    pt = ctypes.cast(ctypes.c_void_p(FAKE), ctypes.POINTER(ctypes.c_int32))
+
+    def append(pool, chunk=0, k=FAKE):
+        return abi.lib.wf_kv_append_fp8(ctypes.byref(pool), 0, chunk, k, FAKE, pt,
+                                        ctypes.byref(desc.c), None)
+
+    def dequant(src, dst, chunk=0):
+        return abi.lib.wf_kv_dequant(ctypes.byref(src), ctypes.byref(dst), 0, chunk, pt,
+                                     ctypes.byref(desc.c), None)
+    assert append(_fp8_pool(abi, k_scale=FAKE + 4)) == abi.WF_ERR_INVALID_ARG    # misaligned
+    assert append(_fp8_pool(abi, v_codes=None)) == abi.WF_ERR_INVALID_ARG
+    assert append(_fp8_pool(abi, head_dim=96)) == abi.WF_ERR_SHAPE
+    assert append(_fp8_pool(abi, page_size=24)) == abi.WF_ERR_SHAPE
+    assert append(_fp8_pool(abi), chunk=3) == abi.WF_ERR_INVALID_ARG             # no such chunk
+    assert append(_fp8_pool(abi), k=FAKE + 2) == abi.WF_ERR_INVALID_ARG
+    short = abi.WavefrontDesc([0, 64, 128, 200], [0, 200, 1000], 1, 2)   # 4 pages needed > 2
+    assert abi.lib.wf_kv_append_fp8(ctypes.byref(_fp8_pool(abi)), 0, 0, FAKE, FAKE, pt,
+                                    ctypes.byref(short.c), None) == abi.WF_ERR_CAPACITY
+    assert dequant(_fp8_pool(abi), _pool(abi, num_heads=3)) == abi.WF_ERR_SHAPE  # geometries differ
+    assert dequant(_fp8_pool(abi), _pool(abi, k_pool=FAKE + 8)) == abi.WF_ERR_INVALID_ARG
+    empty = abi.WavefrontDesc([0, 64, 64], [0, 0], 1, 8)
+    assert abi.lib.wf_kv_append_fp8(ctypes.byref(_fp8_pool(abi)), 0, 1, FAKE, FAKE, pt,
+                                    ctypes.byref(empty.c), None) == abi.WF_OK      # empty chunk
+    if not torch.cuda.is_available():
+        assert append(_fp8_pool(abi)) == abi.WF_ERR_NO_DEVICE
+        assert dequant(_fp8_pool(abi), _pool(abi)) == abi.WF_ERR_NO_DEVICE
