@@ -249,13 +249,16 @@ def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
                hbm_peak: float) -> dict:
     """The FP8 transport kernels over every chunk of the workload's layer: wf_kv_append_fp8
     (bf16 rows -> e4m3 pages + per-(token, head) scales) and wf_kv_dequant (back into the bf16
-    pool), each leg timed with CUDA events on the launching stream after a 256 MB write that
-    flushes L2.  Algorithmic bytes: every K/V element read once and written once."""
+    pool), each leg timed with CUDA events on the launching stream after a 256 MB read that
+    evicts L2.  The read writes back whatever the previous leg left dirty, outside the timed
+    region, and leaves L2 holding clean lines only.  Algorithmic bytes: every K/V element read
+    once in one format and written once in the other."""
     import block_causal_streaming_b200 as wf
     from block_causal_streaming_b200.layer import PagedPoolFp8
     H, D, off = wl.heads, wl.head_dim, wl.chunk_offsets
     fp = PagedPoolFp8(wl.num_pages, wl.page_size, H, D, dev)
-    flush = torch.empty(64 * 2 ** 20, dtype=torch.float32, device=dev)      # 256 MB > L2
+    flush = torch.ones(64 * 2 ** 20, dtype=torch.float32, device=dev)       # 256 MB > L2
+    sink = torch.empty((), dtype=torch.float32, device=dev)
     chunks = range(wl.num_chunks)
 
     def quant():
@@ -274,11 +277,11 @@ def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     torch.cuda.synchronize(dev)
     for e in evs:
-        flush.zero_()
+        torch.sum(flush, out=sink)
         e[0].record(stream)
         quant()
         e[1].record(stream)
-        flush.zero_()
+        torch.sum(flush, out=sink)
         e[2].record(stream)
         dequant()
         e[3].record(stream)
