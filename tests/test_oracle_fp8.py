@@ -96,3 +96,22 @@ def test_dequantized_rows_are_the_bf16_rounding_of_the_fp32_product():
     prod = fp8.e4m3_decode(codes).astype(np.float64) * scale.astype(np.float64)[:, None]
     # nearest bf16 of the product: within half a bf16 ulp (8 significand bits: 2^-8 relative)
     assert np.all(np.abs(got - prod) <= np.abs(prod) * 2.0 ** -8 + 1e-38)
+
+
+def test_attention_over_fp8_kv_stays_near_the_bf16_result():
+    """What FP8 transport costs in attention accuracy, oracle against oracle.  The measured cost is
+    max-abs 0.053 and mean-abs 0.0047 on the tiny workload with N(0,1) values.  That is above the
+    bf16 parity bar, so GPU parity for FP8 pages is defined on the dequantized K/V.  The bound here
+    guards against an encoding that loses much more."""
+    import math
+
+    import oracle
+    from block_causal_streaming_b200.workloads import TINY, make_inputs
+    inp = make_inputs(TINY)
+    k8, v8 = (fp8.dequantize_rows(*fp8.quantize_rows(x.float().numpy())) for x in (inp.k, inp.v))
+    scale = 1.0 / math.sqrt(TINY.head_dim)
+    ref = oracle.attention(inp.q, inp.k, inp.v, TINY.chunk_offsets, TINY.num_ctx_chunks, scale)
+    got = oracle.attention(inp.q, k8, v8, TINY.chunk_offsets, TINY.num_ctx_chunks, scale)
+    err = np.abs(got - ref)
+    assert err.max() <= 0.1 and err.mean() <= 0.01
+    assert err.mean() > 1e-4            # the quantization really happened
