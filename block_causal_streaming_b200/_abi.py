@@ -159,6 +159,53 @@ def _stream_handle(stream) -> Optional[int]:
     return getattr(stream, "cuda_stream", stream)
 
 
+# ---- shapes.  The C ABI takes plain pointers and cannot see a buffer's size, so these checks
+# are what keeps a wrongly shaped tensor from being read or written past its end on the device.
+def _pool_shape(k_pool, v_pool, what: str = "pool"):
+    if k_pool.dim() != 4 or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError(f"{what}: K and V must both be [num_pages, page_size, H, D], got "
+                         f"{tuple(k_pool.shape)} and {tuple(v_pool.shape)}")
+    return tuple(int(x) for x in k_pool.shape)
+
+
+def _check_chunk_rows(wf: "WavefrontDesc", chunk: int, k, v, H: int, D: int):
+    off = wf.chunk_offsets
+    if not 0 <= int(chunk) < len(off) - 1:
+        return                                     # the library answers WF_ERR_INVALID_ARG
+    want = (off[chunk + 1] - off[chunk], H, D)
+    for t, n in ((k, "k"), (v, "v")):
+        if tuple(t.shape) != want and not (want[0] == 0 and t.numel() == 0):
+            raise ValueError(f"{n}: chunk {chunk} needs [{want[0]}, {H}, {D}], got {tuple(t.shape)}")
+
+
+def _check_page_table(page_table, layer: int, wf: "WavefrontDesc"):
+    if page_table.dim() != 2 or page_table.shape[1] != wf.c.max_pages_per_seq:
+        raise ValueError(f"page_table: expected [num_layers, {wf.c.max_pages_per_seq}], got "
+                         f"{tuple(page_table.shape)}")
+    if not 0 <= int(layer) < page_table.shape[0]:
+        raise ValueError(f"layer {layer} outside the page table's {page_table.shape[0]} rows")
+
+
+def _check_page_table_row(row, wf: "WavefrontDesc"):
+    if row.dim() != 1 or row.shape[0] < wf.c.max_pages_per_seq:
+        raise ValueError(f"page_table_row: expected [{wf.c.max_pages_per_seq}], got "
+                         f"{tuple(row.shape)}")
+
+
+def _check_queries(q, out, lse, wf: "WavefrontDesc", H: int, D: int):
+    off = wf.chunk_offsets
+    t_q = off[-1] - off[wf.num_ctx_chunks] if 0 <= wf.num_ctx_chunks < len(off) else None
+    if t_q is None:
+        return                                     # the library answers WF_ERR_SHAPE
+    if tuple(q.shape) != (t_q, H, D):
+        raise ValueError(f"q: expected [{t_q}, {H}, {D}] (the query chunks' rows), got "
+                         f"{tuple(q.shape)}")
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError(f"out: expected {tuple(q.shape)}, got {tuple(out.shape)}")
+    if lse is not None and tuple(lse.shape) != (H, t_q):
+        raise ValueError(f"lse: expected [{H}, {t_q}], got {tuple(lse.shape)}")
+
+
 def _check_tensor(t, name: str, dtype_name: str):
     import torch
     want = {"bf16": (torch.bfloat16,), "i32": (torch.int32,), "f32": (torch.float32,),
@@ -176,6 +223,9 @@ def kv_append(k_pool, v_pool, layer: int, chunk: int, k, v, page_table, wf: Wave
               stream=None) -> None:
     """wf_kv_append: write chunk ``chunk``'s K/V ([L, H, D] bf16) into the pools' pages using row
     ``layer`` of ``page_table`` ([num_layers, max_pages_per_seq] int32, on the device)."""
+    _, _, H, D = _pool_shape(k_pool, v_pool)
+    _check_chunk_rows(wf, chunk, k, v, H, D)
+    _check_page_table(page_table, layer, wf)
     for t, n, d in ((k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"), (k, "k", "bf16"),
                     (v, "v", "bf16"), (page_table, "page_table", "i32")):
         _check_tensor(t, n, d)
@@ -188,15 +238,19 @@ def kv_append(k_pool, v_pool, layer: int, chunk: int, k, v, page_table, wf: Wave
         raise WfError(rc, "wf_kv_append")
 
 
+def _fp8_pool_shape(k_codes, v_codes, k_scale, v_scale):
+    num_pages, page_size, H, D = _pool_shape(k_codes, v_codes, "FP8 pool codes")
+    if tuple(k_scale.shape) != (num_pages, page_size, H) or \
+            tuple(v_scale.shape) != (num_pages, page_size, H):
+        raise ValueError("FP8 pool: codes [pages, page_size, H, D] and scales [pages, page_size, H]")
+    return num_pages, page_size, H, D
+
+
 def _fp8_pool_struct(k_codes, v_codes, k_scale, v_scale) -> KvPoolFp8:
-    num_pages, page_size, H, D = (int(x) for x in k_codes.shape)
+    num_pages, page_size, H, D = _fp8_pool_shape(k_codes, v_codes, k_scale, v_scale)
     for t, n, d in ((k_codes, "k_codes", "u8"), (v_codes, "v_codes", "u8"),
                     (k_scale, "k_scale", "f32"), (v_scale, "v_scale", "f32")):
         _check_tensor(t, n, d)
-    if tuple(v_codes.shape) != tuple(k_codes.shape) or \
-            tuple(k_scale.shape) != (num_pages, page_size, H) or \
-            tuple(v_scale.shape) != (num_pages, page_size, H):
-        raise ValueError("FP8 pool: codes [pages, page_size, H, D] and scales [pages, page_size, H]")
     return KvPoolFp8(k_codes.data_ptr(), v_codes.data_ptr(), k_scale.data_ptr(),
                      v_scale.data_ptr(), num_pages, page_size, H, D)
 
@@ -205,6 +259,9 @@ def kv_append_fp8(k_codes, v_codes, k_scale, v_scale, layer: int, chunk: int, k,
                   wf: WavefrontDesc, stream=None) -> None:
     """wf_kv_append_fp8: quantize chunk ``chunk``'s K/V ([L, H, D] bf16) to e4m3 codes with one
     fp32 scale per (token, head) row, into an FP8 pool through row ``layer`` of ``page_table``."""
+    _, _, H, D = _fp8_pool_shape(k_codes, v_codes, k_scale, v_scale)
+    _check_chunk_rows(wf, chunk, k, v, H, D)
+    _check_page_table(page_table, layer, wf)
     for t, n, d in ((k, "k", "bf16"), (v, "v", "bf16"), (page_table, "page_table", "i32")):
         _check_tensor(t, n, d)
     pool = _fp8_pool_struct(k_codes, v_codes, k_scale, v_scale)
@@ -219,6 +276,10 @@ def kv_append_fp8(k_codes, v_codes, k_scale, v_scale, layer: int, chunk: int, k,
 def kv_dequant(k_codes, v_codes, k_scale, v_scale, k_pool, v_pool, layer: int, chunk: int,
                page_table, wf: WavefrontDesc, stream=None) -> None:
     """wf_kv_dequant: chunk ``chunk`` of an FP8 pool -> the same rows of a bf16 pool."""
+    geo = _fp8_pool_shape(k_codes, v_codes, k_scale, v_scale)
+    if _pool_shape(k_pool, v_pool) != geo:
+        raise ValueError(f"bf16 pool {tuple(k_pool.shape)} differs from the FP8 pool {geo}")
+    _check_page_table(page_table, layer, wf)
     for t, n, d in ((k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
                     (page_table, "page_table", "i32")):
         _check_tensor(t, n, d)
@@ -236,6 +297,9 @@ def attn_forward(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: fl
                  lse=None, stream=None) -> None:
     """wf_attn_forward: block-causal chunk attention of q ([T_q, H, D] bf16) over the paged K/V
     of one layer (``page_table_row``: [max_pages_per_seq] int32 on the device) into ``out``."""
+    _, _, H, D = _pool_shape(k_pool, v_pool)
+    _check_queries(q, out, lse, wf, H, D)
+    _check_page_table_row(page_table_row, wf)
     for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
                     (page_table_row, "page_table_row", "i32"), (out, "out", "bf16")):
         _check_tensor(t, n, d)
@@ -264,6 +328,9 @@ def attn_forward_split(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, sca
     """wf_attn_forward_split: attn_forward with every unit's keys split over ``splits`` CTAs
     (0: the library chooses) and merged; ``workspace`` is a device uint8 tensor of at least
     attn_workspace_size(...) bytes (None when that is 0)."""
+    _, _, H, D = _pool_shape(k_pool, v_pool)
+    _check_queries(q, out, lse, wf, H, D)
+    _check_page_table_row(page_table_row, wf)
     for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
                     (page_table_row, "page_table_row", "i32"), (out, "out", "bf16")):
         _check_tensor(t, n, d)
@@ -287,6 +354,9 @@ def attn_forward_split_noalloc(q, k_pool, v_pool, page_table_row, wf: WavefrontD
                                scale: float, out, splits: int = 0, lse=None, stream=None) -> None:
     """wf_attn_forward_split_noalloc: attn_forward_split with the library's static scratch
     instead of a workspace (calls on one device must be ordered on one stream)."""
+    _, _, H, D = _pool_shape(k_pool, v_pool)
+    _check_queries(q, out, lse, wf, H, D)
+    _check_page_table_row(page_table_row, wf)
     for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
                     (page_table_row, "page_table_row", "i32"), (out, "out", "bf16")):
         _check_tensor(t, n, d)
@@ -309,6 +379,12 @@ def kv_append_publish(k_pool, v_pool, flags, peers, layer: int, chunk: int, k, v
     """wf_kv_append_publish: append one chunk into this pool and every peer pool, then raise the
     chunk's flag to ``generation`` here (``flags``: device uint32 [layers, WF_MAX_CHUNKS] or
     None) and in every peer.  ``peers``: sequence of (k_pool_ptr, v_pool_ptr, flags_ptr)."""
+    _, _, H, D = _pool_shape(k_pool, v_pool)
+    _check_chunk_rows(wf, chunk, k, v, H, D)
+    _check_page_table(page_table, layer, wf)
+    if flags is not None and flags.numel() < (int(layer) + 1) * WF_MAX_CHUNKS:
+        raise ValueError(f"flags: layer {layer} needs [>= {int(layer) + 1}, {WF_MAX_CHUNKS}] words, "
+                         f"got {tuple(flags.shape)}")
     for t, n, d in ((k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
                     (page_table, "page_table", "i32")):
         _check_tensor(t, n, d)
@@ -335,6 +411,11 @@ def attn_forward_published(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc,
                            lse=None, stream=None) -> None:
     """wf_attn_forward_published: attn_forward_split that waits, chunk by chunk, for the
     publication flags in ``flags_row`` (device uint32 [WF_MAX_CHUNKS]) to reach ``generation``."""
+    _, _, H, D = _pool_shape(k_pool, v_pool)
+    _check_queries(q, out, lse, wf, H, D)
+    _check_page_table_row(page_table_row, wf)
+    if flags_row.numel() < len(wf.chunk_offsets) - 1:
+        raise ValueError(f"flags_row: one word per chunk needed, got {tuple(flags_row.shape)}")
     for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
                     (page_table_row, "page_table_row", "i32"), (out, "out", "bf16"),
                     (flags_row, "flags_row", "u32")):
