@@ -29,7 +29,7 @@ EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror",
             "wf_selftest_timeout", "wf_attn_forward_split", "wf_attn_workspace_size",
             "wf_attn_forward_split_noalloc", "wf_kv_append_publish", "wf_attn_forward_published",
             "wf_ipc_export", "wf_ipc_import", "wf_ipc_close", "wf_kv_append_fp8",
-            "wf_kv_dequant")
+            "wf_kv_dequant", "wf_window_slots", "wf_window_round")
 
 
 class WfError(RuntimeError):
@@ -56,6 +56,21 @@ class KvPoolFp8(ctypes.Structure):
                 ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
                 ("num_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
                 ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+class WindowC(ctypes.Structure):
+    """wf_window_t."""
+    _fields_ = [("chunk_len", ctypes.c_int32), ("num_stages", ctypes.c_int32),
+                ("stages", ctypes.POINTER(ctypes.c_int32)), ("history", ctypes.c_int32)]
+
+
+class RoundC(ctypes.Structure):
+    """wf_round_t."""
+    _fields_ = [("round", ctypes.c_int64), ("num_chunks", ctypes.c_int32),
+                ("num_ctx_chunks", ctypes.c_int32), ("chunk_id", ctypes.c_int64 * 64),
+                ("role", ctypes.c_int32 * 64), ("chunk_stage", ctypes.c_int32 * 64),
+                ("chunk_offsets", ctypes.c_int32 * 65), ("store_to", ctypes.c_int32),
+                ("evicted", ctypes.c_int64)]
 
 
 class Wavefront(ctypes.Structure):
@@ -121,6 +136,12 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wf_kv_dequant.argtypes = [ctypes.POINTER(KvPoolFp8), ctypes.POINTER(KvPool), i32, i32,
                                   ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(Wavefront), vp]
     lib.wf_kv_dequant.restype = i32
+    lib.wf_window_slots.argtypes = [ctypes.POINTER(WindowC), ctypes.POINTER(ctypes.c_int32),
+                                    ctypes.POINTER(ctypes.c_int64)]
+    lib.wf_window_slots.restype = i32
+    lib.wf_window_round.argtypes = [ctypes.POINTER(WindowC), ctypes.c_int64,
+                                    ctypes.POINTER(RoundC)]
+    lib.wf_window_round.restype = i32
     return lib
 
 
@@ -217,6 +238,33 @@ def _check_tensor(t, name: str, dtype_name: str):
         raise ValueError(f"{name}: expected a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name}: expected a contiguous tensor")
+
+
+class Window:
+    """Host copy of a wf_window_t; keeps the stage array alive while C reads it."""
+
+    def __init__(self, chunk_len: int, stages: Sequence[int], history: int):
+        self._stages = (ctypes.c_int32 * max(len(stages), 1))(*[int(s) for s in stages])
+        self.c = WindowC(int(chunk_len), len(stages),
+                         ctypes.cast(self._stages, ctypes.POINTER(ctypes.c_int32)), int(history))
+
+
+def window_slots(window: Window):
+    """wf_window_slots: (slots, tokens) of one layer of the window."""
+    slots, tokens = ctypes.c_int32(), ctypes.c_int64()
+    rc = lib.wf_window_slots(ctypes.byref(window.c), ctypes.byref(slots), ctypes.byref(tokens))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_window_slots")
+    return slots.value, tokens.value
+
+
+def window_round(window: Window, round_index: int) -> RoundC:
+    """wf_window_round: the plan of one round."""
+    out = RoundC()
+    rc = lib.wf_window_round(ctypes.byref(window.c), int(round_index), ctypes.byref(out))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_window_round")
+    return out
 
 
 def kv_append(k_pool, v_pool, layer: int, chunk: int, k, v, page_table, wf: WavefrontDesc,

@@ -2,8 +2,10 @@
 
     python -m block_causal_streaming_b200.build [-v]
 
-The library is one translation unit (``csrc/wf_api.cu``, which includes the kernels) linked
-against the static CUDA runtime, so it only needs the driver at run time.
+The library is two translation units linked against the static CUDA runtime, so it only needs
+the driver at run time:
+- ``csrc/wf_api.cu`` includes the kernels;
+- ``csrc/wf_window.cpp`` is the host-only rolling-window planner.
 """
 from __future__ import annotations
 
@@ -16,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libwf_b200.so")
-SOURCES = [os.path.join(CSRC, "wf_api.cu")]
+SOURCES = [os.path.join(CSRC, "wf_api.cu"), os.path.join(CSRC, "wf_window.cpp")]
 DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "attn_kernel.cuh",
                                                       "attn_pair_kernel.cuh",
                                                       "append_kernel.cuh", "combine_kernel.cuh",

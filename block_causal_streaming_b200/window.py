@@ -38,7 +38,7 @@ cannot be moved by editing page-table entries.  Nothing that persists is moved, 
   leaves (``RoundView.store_to``).  That is one extra chunk append per layer per round.
 
 :class:`RollingWindow` is the host-side planner: a pure function from the round number to that
-round's descriptor.  :class:`RollingCache` holds the device pools and page tables.  Through the C
+round's descriptor, computed by the library's native planner (``wf_window_round``).  :class:`RollingCache` holds the device pools and page tables.  Through the C
 ABI it runs one layer of a round: appends, attention and the hand-over into the ring.
 """
 from __future__ import annotations
@@ -50,7 +50,8 @@ from typing import List, Optional, Sequence
 import torch
 
 ANCHOR, HISTORY, STORE, ACTIVE = "anchor", "history", "store", "active"
-MAX_CHUNKS = 64   # chunks per descriptor (WF_MAX_CHUNKS); the planner runs without the library
+_ROLE_NAMES = {0: ANCHOR, 1: HISTORY, 2: STORE, 3: ACTIVE}   # WF_ROLE_* of include/wf.h
+MAX_CHUNKS = 64   # chunks per descriptor (WF_MAX_CHUNKS)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -95,73 +96,43 @@ class RoundView:
 
 
 class RollingWindow:
-    """Round-by-round plan of a streaming wavefront with a rolling history.
+    """Round-by-round plan of a streaming wavefront with a rolling history (wf_window_round).
 
     ``stages`` are the denoising timesteps of the in-flight positions, noisiest first (e.g.
     1000, 800, 600, 400, 200).  Chunk ``c`` enters at round ``c``.  At round ``t`` it is on step
-    ``t - c``, and in the store pass at round ``c + len(stages)``.
+    ``t - c``, and in the store pass at round ``c + len(stages)``.  The plan comes from the
+    library's native planner; this class only converts it.
     """
 
     def __init__(self, chunk_len: int, stages: Sequence[int], history: int, page_size: int):
-        stages = [int(s) for s in stages]
-        if chunk_len < 1 or history < 0 or not stages:
-            raise ValueError("chunk_len >= 1, history >= 0 and at least one stage are required")
-        if any(s <= 0 for s in stages) or any(a <= b for a, b in zip(stages, stages[1:])):
-            raise ValueError("stages must be positive and strictly decreasing (noisiest first)")
+        from . import _abi
         self.chunk_len = int(chunk_len)
-        self.stages = stages
+        self.stages = [int(x) for x in stages]
         self.history = int(history)
         self.page_size = int(page_size)
-        self.slots = 1 + self.history + 1 + len(stages)
-        if self.slots > MAX_CHUNKS:
-            raise ValueError(f"{self.slots} chunk slots exceed the descriptor's {MAX_CHUNKS}")
-        self.tokens = self.slots * self.chunk_len
+        if not self.stages or self.page_size < 1:
+            raise ValueError("at least one stage and a positive page size are required")
+        self._w = _abi.Window(self.chunk_len, self.stages, self.history)
+        try:
+            self.slots, self.tokens = _abi.window_slots(self._w)
+        except _abi.WfError as e:
+            raise ValueError(f"invalid window (chunk_len >= 1, history >= 0, stages positive and "
+                             f"strictly decreasing, at most {MAX_CHUNKS} slots): {e}") from None
         self.pages = math.ceil(self.tokens / self.page_size)
 
-    def ring_slot(self, chunk_id: int) -> int:
-        """Slot kept by a stored chunk: 0 for the anchor, then the ring."""
-        if chunk_id == 0:
-            return 0
-        if self.history == 0:
-            raise ValueError("no history is kept")
-        return 1 + (chunk_id - 1) % self.history
-
     def view(self, t: int) -> RoundView:
+        from . import _abi
         if t < 0:
             raise ValueError("rounds start at 0")
-        S, W, L = len(self.stages), self.history, self.chunk_len
-        last_stored = t - S - 1                      # chunks <= this finished their store pass
-        ids: List[int] = []
-        roles: List[str] = []
-        stage: List[int] = []
-        if last_stored >= 0:
-            ids.append(0)
-            roles.append(ANCHOR)
-            stage.append(0)
-            kept = list(range(max(1, last_stored - W + 1), last_stored + 1)) if W > 0 else []
-            by_slot = sorted(kept, key=self.ring_slot)
-            ids += by_slot
-            roles += [HISTORY] * len(by_slot)
-            stage += [0] * len(by_slot)
-        n_ctx = len(ids)
-        store = t - S
-        store_to = evicted = None
-        if store >= 0:
-            ids.append(store)
-            roles.append(STORE)
-            stage.append(0)
-            if store >= 1 and W > 0 and store - W >= 1:
-                # the ring is full: the store chunk takes the slot of the chunk that leaves
-                evicted = store - W
-                store_to = self.ring_slot(store)
-        for c in range(max(0, t - S + 1), t + 1):     # in flight, oldest (cleanest) first
-            ids.append(c)
-            roles.append(ACTIVE)
-            stage.append(self.stages[t - c])
-        offsets = [i * L for i in range(len(ids) + 1)]
-        return RoundView(round=t, chunk_ids=ids, roles=roles, chunk_stage=stage,
-                         chunk_offsets=offsets, num_ctx_chunks=n_ctx, store_to=store_to,
-                         evicted=evicted)
+        r = _abi.window_round(self._w, t)
+        n = r.num_chunks
+        return RoundView(round=int(r.round), chunk_ids=[int(x) for x in r.chunk_id[:n]],
+                         roles=[_ROLE_NAMES[x] for x in r.role[:n]],
+                         chunk_stage=[int(x) for x in r.chunk_stage[:n]],
+                         chunk_offsets=[int(x) for x in r.chunk_offsets[:n + 1]],
+                         num_ctx_chunks=int(r.num_ctx_chunks),
+                         store_to=None if r.store_to < 0 else int(r.store_to),
+                         evicted=None if r.evicted < 0 else int(r.evicted))
 
 
 class RollingCache:

@@ -277,6 +277,72 @@ int wf_kv_dequant(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int laye
                   const int32_t* page_table, const wf_wavefront_t* wf, wf_stream_t stream);
 
 /*
+ * Rolling context window: the plan of one round of a stream (host only, no device work).
+ *
+ * The pages' rules:
+ *   - Round t of a stream has its active cells on a diagonal that advances one chunk per round:
+ *     chunk c enters at round c, is on denoising step t - c at round t, and gets its store pass
+ *     (a forward pass at the clean timestep whose K/V become history) at round c + num_stages.
+ *   - A chunk sees the anchor, the clean history, the live store and every earlier, cleaner chunk
+ *     in flight, and never a later, noisier one (KipQuest summary of arXiv 2611.00859, "The deep
+ *     dive").
+ *
+ * Readings taken here:
+ *   - The anchor is the first chunk stored; it is kept for the whole stream.
+ *   - The history is the `history` most recently stored chunks after the anchor.
+ *   - Every chunk has chunk_len tokens.
+ *
+ * Layout.  Every layer uses one fixed page table over
+ * slots = 1 + history + 1 + num_stages chunk slots of chunk_len tokens:
+ *   [anchor][history ring][live store][in flight, cleanest first].
+ *
+ * Order and placement:
+ *   - Anchor and history keep their slots.  Every query sees all of them, so their order does not
+ *     matter, and the history is a ring: slot 1 + (c - 1) mod history for stored chunk c >= 1.
+ *   - The store chunk and the chunks in flight are appended every round right after the last
+ *     occupied history slot.
+ *   - While the ring fills, the store chunk already sits in its own ring slot.
+ *   - Once the ring is full, the store chunk's K/V must also be appended into slot `store_to` (the
+ *     slot of the chunk that leaves, `evicted`) after the round's attention at that layer.
+ *
+ * Slot i holds logical tokens [i * chunk_len, (i + 1) * chunk_len), so a round's chunk_offsets and
+ * chunk_stage can be passed straight into a wf_wavefront_t (num_chunks, num_ctx_chunks likewise).
+ */
+enum { WF_ROLE_ANCHOR = 0, WF_ROLE_HISTORY = 1, WF_ROLE_STORE = 2, WF_ROLE_ACTIVE = 3 };
+
+typedef struct {
+  int32_t chunk_len;        /* tokens per chunk, >= 1 */
+  int32_t num_stages;       /* denoising steps = in-flight positions, >= 1 */
+  const int32_t* stages;    /* host [num_stages]: timesteps, noisiest first, > 0, strictly decreasing */
+  int32_t history;          /* clean-history chunks kept after the anchor, >= 0 */
+} wf_window_t;
+
+typedef struct {
+  int64_t round;
+  int32_t num_chunks;                          /* occupied slots, in logical order */
+  int32_t num_ctx_chunks;                      /* anchor + history: K/V only this round */
+  int64_t chunk_id[WF_MAX_CHUNKS];             /* stream index of the chunk in each slot */
+  int32_t role[WF_MAX_CHUNKS];                 /* WF_ROLE_* */
+  int32_t chunk_stage[WF_MAX_CHUNKS];          /* 0 for anchor, history, store */
+  int32_t chunk_offsets[WF_MAX_CHUNKS + 1];
+  int32_t store_to;                            /* slot for the store hand-over, or -1 */
+  int64_t evicted;                             /* chunk leaving the history after the round, or -1 */
+} wf_round_t;
+
+/*
+ * wf_window_slots -- slots and tokens one layer of the window occupies (pages needed:
+ * ceil(tokens / page_size)).  WF_ERR_INVALID_ARG for null pointers, WF_ERR_SHAPE for a window that
+ * breaks the rules above, needs more than WF_MAX_CHUNKS slots or more than INT32_MAX tokens.
+ */
+int wf_window_slots(const wf_window_t* window, int32_t* slots, int64_t* tokens);
+
+/*
+ * wf_window_round -- the plan of round `round` (>= 0) into *out.  Errors as wf_window_slots;
+ * WF_ERR_INVALID_ARG for a negative round.
+ */
+int wf_window_round(const wf_window_t* window, int64_t round, wf_round_t* out);
+
+/*
  * wf_check_status -- synchronise `stream`, then return and clear the first error any kernel of
  * this library recorded on the current device since the last call (WF_OK if none).  A pending
  * CUDA error on the stream is returned as WF_ERR_CUDA.

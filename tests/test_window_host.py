@@ -10,11 +10,17 @@
   own paged scatter and gather, leave in every slot exactly the chunk the round's descriptor names,
   bit for bit.
 """
+import ctypes
+
 import numpy as np
 import pytest
 
 import oracle
-from block_causal_streaming_b200 import window as W
+from block_causal_streaming_b200 import build as wf_build
+
+wf_build.build()                      # the planner is the library's wf_window_round
+from block_causal_streaming_b200 import _abi  # noqa: E402
+from block_causal_streaming_b200 import window as W  # noqa: E402
 
 SHAPES = [(1, 0), (1, 2), (2, 1), (4, 2), (5, 1), (5, 3), (3, 5)]   # (stages, history)
 
@@ -138,7 +144,59 @@ def test_planner_argument_checks():
 
 
 def test_max_chunks_matches_the_library():
-    from block_causal_streaming_b200 import build as wf_build
-    wf_build.build()
-    from block_causal_streaming_b200 import _abi
     assert W.MAX_CHUNKS == _abi.WF_MAX_CHUNKS
+
+
+def _plan_written_out(chunk_len, stages, history, t):
+    """A second, independent statement of the layout (sorting kept chunks by ring slot), used to
+    cross-check the native planner's slot assignment."""
+    S, H = len(stages), history
+    ring = lambda c: 0 if c == 0 else 1 + (c - 1) % H                       # noqa: E731
+    ids, roles, stage = [], [], []
+    last_stored = t - S - 1
+    if last_stored >= 0:
+        kept = list(range(max(1, last_stored - H + 1), last_stored + 1)) if H else []
+        ids += [0] + sorted(kept, key=ring)
+        roles += [W.ANCHOR] + [W.HISTORY] * len(kept)
+        stage += [0] * (1 + len(kept))
+    n_ctx, store_to, evicted = len(ids), None, None
+    if t - S >= 0:
+        ids.append(t - S)
+        roles.append(W.STORE)
+        stage.append(0)
+        if H and t - S - H >= 1:
+            evicted, store_to = t - S - H, ring(t - S)
+    for c in range(max(0, t - S + 1), t + 1):
+        ids.append(c)
+        roles.append(W.ACTIVE)
+        stage.append(stages[t - c])
+    return ids, roles, stage, n_ctx, store_to, evicted
+
+
+@pytest.mark.parametrize("S,H", SHAPES + [(2, 7), (6, 4), (1, 1), (3, 2), (2, 3)])
+def test_native_planner_matches_the_written_out_layout(S, H):
+    win = W.RollingWindow(33, _stages(S), H, 16)
+    for t in range(0, 4 * (S + H) + 9):
+        v = win.view(t)
+        ids, roles, stage, n_ctx, store_to, evicted = _plan_written_out(33, _stages(S), H, t)
+        assert (v.chunk_ids, v.roles, v.chunk_stage, v.num_ctx_chunks, v.store_to, v.evicted) == \
+            (ids, roles, stage, n_ctx, store_to, evicted), t
+
+
+def test_native_planner_argument_checks():
+    w = _abi.Window(48, [1000, 500], 2)
+    out = _abi.RoundC()
+    assert _abi.lib.wf_window_round(None, 0, ctypes.byref(out)) == _abi.WF_ERR_INVALID_ARG
+    assert _abi.lib.wf_window_round(ctypes.byref(w.c), 0, None) == _abi.WF_ERR_INVALID_ARG
+    assert _abi.lib.wf_window_round(ctypes.byref(w.c), -1, ctypes.byref(out)) == \
+        _abi.WF_ERR_INVALID_ARG
+    assert _abi.window_slots(w) == (5 + 1, 6 * 48)
+    for bad in (_abi.Window(48, [500, 1000], 2), _abi.Window(48, [1000, 0], 2),
+                _abi.Window(0, [1000], 2), _abi.Window(48, [1000], -1),
+                _abi.Window(48, [1000], 62), _abi.Window(2 ** 26, [1000], 62 - 30)):
+        with pytest.raises(_abi.WfError) as e:
+            _abi.window_slots(bad)
+        assert e.value.code == _abi.WF_ERR_SHAPE
+    assert _abi.window_slots(_abi.Window(48, [1000], 61)) == (64, 64 * 48)
+    big = _abi.window_round(w, 10 ** 12)                 # far into a stream: 64-bit chunk ids
+    assert big.chunk_id[big.num_chunks - 1] == 10 ** 12
