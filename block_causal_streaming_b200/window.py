@@ -38,8 +38,9 @@ cannot be moved by editing page-table entries.  Nothing that persists is moved, 
   leaves (``RoundView.store_to``).  That is one extra chunk append per layer per round.
 
 :class:`RollingWindow` is the host-side planner: a pure function from the round number to that
-round's descriptor, computed by the library's native planner (``wf_window_round``).  :class:`RollingCache` holds the device pools and page tables.  Through the C
-ABI it runs one layer of a round: appends, attention and the hand-over into the ring.
+round's descriptor, computed by the library's native planner (``wf_window_round``).
+:class:`RollingCache` holds the device pools and page tables.  Through the C ABI it runs one
+layer of a round: appends, attention and the hand-over into the ring.
 """
 from __future__ import annotations
 
