@@ -32,7 +32,8 @@
  *     errors are detected on the host before anything is launched.  Errors found by a kernel
  *     (a page index outside the pool, a bounded wait that ran out) are recorded in a per-device
  *     status word read by wf_check_status.
- *   - bf16 only, batch 1, one layer per call.
+ *   - Attention computes in bf16 with fp32 accumulation; FP8 appears only in the K/V transport
+ *     calls (wf_kv_append_fp8, wf_kv_dequant).  Batch 1, one layer per call.
  */
 #ifndef WF_H_
 #define WF_H_
