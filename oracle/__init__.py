@@ -35,8 +35,9 @@ _lib = None
 
 
 def build(src: str = _SRC, out: str = _LIB_PATH) -> str:
-    """Compile the C oracle with gcc (plain -O2, no fast-math: IEEE fp64 sums)."""
-    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-fno-fast-math",
+    """Compile the C oracle with gcc (-O3, no fast-math, no FMA contraction: IEEE fp64 sums in
+    the order the source writes them)."""
+    cmd = ["gcc", "-O3", "-ffp-contract=off", "-std=c11", "-fPIC", "-shared", "-pthread", "-fno-fast-math",
            "-o", out, src, "-lm"]
     subprocess.run(cmd, check=True)
     return out

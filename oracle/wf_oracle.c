@@ -55,40 +55,89 @@ static int chunk_of_token(const int32_t *offsets, int num_chunks, int t) {
     return -1;
 }
 
-static void one_row(const job_t *jb, int r, int h, double *s, float *o_out, float *lse_out) {
-    const int H = jb->H, D = jb->D, T_kv = jb->T_kv;
-    const int qc = chunk_of_token(jb->chunk_offsets, jb->num_chunks, jb->T_ctx + r);
-    const float *qr = jb->q + ((size_t)r * H + h) * D;
+/* Whether key j is visible to a query of chunk qc: keys of the same or an earlier chunk only. */
+static int visible(const job_t *jb, int j, int qc) { return jb->key_chunk[j] <= qc; }
+
+/* Key row j and value row j of head h. */
+static const float *key_row(const job_t *jb, int j, int h) {
+    return jb->k + ((size_t)j * jb->H + h) * jb->D;
+}
+static const float *value_row(const job_t *jb, int j, int h) {
+    return jb->v + ((size_t)j * jb->H + h) * jb->D;
+}
+
+/* s[j] = scale * (q_r . k_j), each dot product summed in fp64 in d order.  Four visible keys are
+ * summed side by side (four independent sums, each in the same order as alone); any key of a
+ * later chunk is masked to -inf and its product is never formed.  Returns the largest logit. */
+static double logits(const job_t *jb, const float *qr, int h, int qc, double *s) {
+    const int D = jb->D, T_kv = jb->T_kv;
     double m = -INFINITY;
-    for (int j = 0; j < T_kv; ++j) {
-        if (jb->key_chunk[j] > qc) { s[j] = -INFINITY; continue; }   /* later chunk: masked */
-        const float *kr = jb->k + ((size_t)j * H + h) * D;
+    int j = 0;
+    while (j < T_kv) {
+        if (j + 4 <= T_kv && visible(jb, j, qc) && visible(jb, j + 1, qc) &&
+            visible(jb, j + 2, qc) && visible(jb, j + 3, qc)) {
+            const float *k0 = key_row(jb, j, h), *k1 = key_row(jb, j + 1, h);
+            const float *k2 = key_row(jb, j + 2, h), *k3 = key_row(jb, j + 3, h);
+            double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+            for (int d = 0; d < D; ++d) {
+                const double x = (double)qr[d];
+                a0 += x * (double)k0[d];
+                a1 += x * (double)k1[d];
+                a2 += x * (double)k2[d];
+                a3 += x * (double)k3[d];
+            }
+            const double a[4] = {a0, a1, a2, a3};
+            for (int i = 0; i < 4; ++i) {
+                s[j + i] = jb->scale * a[i];
+                if (s[j + i] > m) m = s[j + i];
+            }
+            j += 4;
+            continue;
+        }
+        if (!visible(jb, j, qc)) { s[j] = -INFINITY; ++j; continue; }   /* later chunk: masked */
+        const float *kr = key_row(jb, j, h);
         double acc = 0.0;
-        for (int d = 0; d < D; ++d) acc += (double)qr[d] * (double)kr[d];
+        for (int d = 0; d < D; ++d) {
+            const double x = (double)qr[d];
+            acc += x * (double)kr[d];
+        }
         s[j] = jb->scale * acc;
         if (s[j] > m) m = s[j];
+        ++j;
     }
+    return m;
+}
+
+/* acc: D doubles of scratch. */
+static void one_row(const job_t *jb, int r, int h, double *s, double *acc, float *o_out,
+                    float *lse_out) {
+    const int D = jb->D, T_kv = jb->T_kv;
+    const int qc = chunk_of_token(jb->chunk_offsets, jb->num_chunks, jb->T_ctx + r);
+    const float *qr = jb->q + ((size_t)r * jb->H + h) * D;
+    const double m = logits(jb, qr, h, qc, s);
     double den = 0.0;
     for (int j = 0; j < T_kv; ++j) {
-        if (jb->key_chunk[j] > qc) { s[j] = 0.0; continue; }
+        if (!visible(jb, j, qc)) { s[j] = 0.0; continue; }
         s[j] = exp(s[j] - m);
         den += s[j];
     }
-    for (int d = 0; d < D; ++d) {
-        double acc = 0.0;
-        for (int j = 0; j < T_kv; ++j) {
-            if (s[j] == 0.0) continue;
-            acc += s[j] * (double)jb->v[((size_t)j * H + h) * D + d];
-        }
-        o_out[d] = (float)(acc / den);
+    /* o[d] = sum_j p_j v[j][d], every column summed over ascending j */
+    for (int d = 0; d < D; ++d) acc[d] = 0.0;
+    for (int j = 0; j < T_kv; ++j) {
+        if (s[j] == 0.0) continue;
+        const float *vr = value_row(jb, j, h);
+        const double p = s[j];
+        for (int d = 0; d < D; ++d) acc[d] += p * (double)vr[d];
     }
+    for (int d = 0; d < D; ++d) o_out[d] = (float)(acc[d] / den);
     if (lse_out) *lse_out = (float)(m + log(den));
 }
 
 static void *worker(void *arg) {
     job_t *jb = (job_t *)arg;
     double *s = (double *)malloc(sizeof(double) * (size_t)(jb->T_kv > 0 ? jb->T_kv : 1));
-    if (!s) return (void *)1;
+    double *acc = (double *)malloc(sizeof(double) * (size_t)jb->D);
+    if (!s || !acc) { free(s); free(acc); return (void *)1; }
     for (;;) {
         int i = __atomic_fetch_add(&jb->next_item, 1, __ATOMIC_RELAXED);
         if (i >= jb->n_items) break;
@@ -105,9 +154,10 @@ static void *worker(void *arg) {
             o = jb->out + ((size_t)r * jb->H + h) * jb->D;
             l = jb->lse ? jb->lse + (size_t)h * jb->T_q + r : NULL;
         }
-        one_row(jb, r, h, s, o, l);
+        one_row(jb, r, h, s, acc, o, l);
     }
     free(s);
+    free(acc);
     return NULL;
 }
 

@@ -20,22 +20,22 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "wf_oracle.c")
 
 # (name, text to find, replacement); every occurrence is replaced; all edits stay in bounds.
 MUTANTS = [
-    ("own_chunk_excluded", "jb->key_chunk[j] > qc", "jb->key_chunk[j] >= qc"),
-    ("mask_reversed", "jb->key_chunk[j] > qc", "jb->key_chunk[j] < qc"),
-    ("no_mask", "jb->key_chunk[j] > qc", "jb->key_chunk[j] > 1000000"),
+    ("own_chunk_excluded", "jb->key_chunk[j] <= qc", "jb->key_chunk[j] < qc"),
+    ("mask_reversed", "jb->key_chunk[j] <= qc", "jb->key_chunk[j] >= qc"),
+    ("no_mask", "jb->key_chunk[j] <= qc", "jb->key_chunk[j] <= 1000000"),
     ("boundary_off_by_one", "t >= offsets[c] && t < offsets[c + 1]",
      "t >= offsets[c] && t <= offsets[c + 1]"),
     ("query_chunk_from_query_index", "jb->T_ctx + r", "r"),
-    ("scale_dropped", "s[j] = jb->scale * acc;", "s[j] = acc;"),
-    ("normalisation_dropped", "o_out[d] = (float)(acc / den);", "o_out[d] = (float)(acc);"),
+    ("scale_dropped", "jb->scale * ", "1.0 * "),
+    ("normalisation_dropped", "o_out[d] = (float)(acc[d] / den);", "o_out[d] = (float)(acc[d]);"),
     ("exp_sign_flipped", "s[j] = exp(s[j] - m);", "s[j] = exp(m - s[j]);"),
-    ("key_head_wrong", "const float *kr = jb->k + ((size_t)j * H + h) * D;",
-     "const float *kr = jb->k + ((size_t)j * H + (h + 1) % H) * D;"),
-    ("value_head_wrong", "(double)jb->v[((size_t)j * H + h) * D + d]",
-     "(double)jb->v[((size_t)j * H + 0) * D + d]"),
-    ("value_row_wrong", "(double)jb->v[((size_t)j * H + h) * D + d]",
-     "(double)jb->v[((size_t)(T_kv - 1 - j) * H + h) * D + d]"),
-    ("query_dim_transposed", "(double)qr[d] * (double)kr[d]", "(double)qr[D - 1 - d] * (double)kr[d]"),
+    ("key_head_wrong", "return jb->k + ((size_t)j * jb->H + h) * jb->D;",
+     "return jb->k + ((size_t)j * jb->H + (h + 1) % jb->H) * jb->D;"),
+    ("value_head_wrong", "return jb->v + ((size_t)j * jb->H + h) * jb->D;",
+     "return jb->v + ((size_t)j * jb->H + 0) * jb->D;"),
+    ("value_row_wrong", "value_row(jb, j, h)", "value_row(jb, T_kv - 1 - j, h)"),
+    ("query_dim_transposed", "const double x = (double)qr[d];",
+     "const double x = (double)qr[D - 1 - d];"),
     ("lse_max_dropped", "*lse_out = (float)(m + log(den));", "*lse_out = (float)(log(den));"),
 ]
 
