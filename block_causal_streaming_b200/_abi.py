@@ -29,7 +29,8 @@ EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror",
             "wf_selftest_timeout", "wf_attn_forward_split", "wf_attn_workspace_size",
             "wf_attn_forward_split_noalloc", "wf_kv_append_publish", "wf_attn_forward_published",
             "wf_ipc_export", "wf_ipc_import", "wf_ipc_close", "wf_kv_append_fp8",
-            "wf_kv_dequant", "wf_window_slots", "wf_window_round")
+            "wf_kv_dequant", "wf_kv_append_publish_fp8", "wf_kv_dequant_published",
+            "wf_window_slots", "wf_window_round")
 
 
 class WfError(RuntimeError):
@@ -41,6 +42,13 @@ class WfError(RuntimeError):
 class PoolDst(ctypes.Structure):
     """wf_pool_dst_t: a destination pool (usually another GPU's, mapped by ipc_import)."""
     _fields_ = [("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p),
+                ("flags", ctypes.c_void_p)]
+
+
+class Fp8Dst(ctypes.Structure):
+    """wf_fp8_dst_t: a destination FP8 pool (usually another GPU's, mapped by ipc_import)."""
+    _fields_ = [("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
+                ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
                 ("flags", ctypes.c_void_p)]
 
 
@@ -136,6 +144,15 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wf_kv_dequant.argtypes = [ctypes.POINTER(KvPoolFp8), ctypes.POINTER(KvPool), i32, i32,
                                   ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(Wavefront), vp]
     lib.wf_kv_dequant.restype = i32
+    lib.wf_kv_append_publish_fp8.argtypes = [ctypes.POINTER(KvPoolFp8), vp,
+                                             ctypes.POINTER(Fp8Dst), i32, i32, i32, vp, vp,
+                                             ctypes.POINTER(ctypes.c_int32),
+                                             ctypes.POINTER(Wavefront), ctypes.c_uint32, vp]
+    lib.wf_kv_append_publish_fp8.restype = i32
+    lib.wf_kv_dequant_published.argtypes = [ctypes.POINTER(KvPoolFp8), ctypes.POINTER(KvPool),
+                                            i32, i32, ctypes.POINTER(ctypes.c_int32),
+                                            ctypes.POINTER(Wavefront), vp, ctypes.c_uint32, vp]
+    lib.wf_kv_dequant_published.restype = i32
     lib.wf_window_slots.argtypes = [ctypes.POINTER(WindowC), ctypes.POINTER(ctypes.c_int32),
                                     ctypes.POINTER(ctypes.c_int64)]
     lib.wf_window_slots.restype = i32
@@ -339,6 +356,65 @@ def kv_dequant(k_codes, v_codes, k_scale, v_scale, k_pool, v_pool, layer: int, c
                            ctypes.byref(wf.c), _stream_handle(stream))
     if rc != WF_OK:
         raise WfError(rc, "wf_kv_dequant")
+
+
+def kv_append_publish_fp8(k_codes, v_codes, k_scale, v_scale, flags, peers, layer: int,
+                          chunk: int, k, v, page_table, wf: WavefrontDesc, generation: int,
+                          stream=None) -> None:
+    """wf_kv_append_publish_fp8: quantize one chunk into this FP8 pool and every peer FP8 pool,
+    then raise the chunk's flag to ``generation`` here (``flags``: device uint32
+    [layers, WF_MAX_CHUNKS] or None) and in every peer.  ``peers``: sequence of
+    (k_codes_ptr, v_codes_ptr, k_scale_ptr, v_scale_ptr, flags_ptr)."""
+    _, _, H, D = _fp8_pool_shape(k_codes, v_codes, k_scale, v_scale)
+    _check_chunk_rows(wf, chunk, k, v, H, D)
+    _check_page_table(page_table, layer, wf)
+    if flags is not None and flags.numel() < (int(layer) + 1) * WF_MAX_CHUNKS:
+        raise ValueError(f"flags: layer {layer} needs [>= {int(layer) + 1}, {WF_MAX_CHUNKS}] words, "
+                         f"got {tuple(flags.shape)}")
+    _check_tensor(page_table, "page_table", "i32")
+    if k.numel() > 0:
+        _check_tensor(k, "k", "bf16")
+        _check_tensor(v, "v", "bf16")
+    if flags is not None:
+        _check_tensor(flags, "flags", "u32")
+    arr = (Fp8Dst * max(1, len(peers)))(*[Fp8Dst(int(a), int(b), int(c), int(d),
+                                                 int(f) if f else None)
+                                          for a, b, c, d, f in peers])
+    pool = _fp8_pool_struct(k_codes, v_codes, k_scale, v_scale)
+    rc = lib.wf_kv_append_publish_fp8(
+        ctypes.byref(pool), flags.data_ptr() if flags is not None else None, arr, len(peers),
+        int(layer), int(chunk), k.data_ptr() if k.numel() else None,
+        v.data_ptr() if v.numel() else None,
+        ctypes.cast(ctypes.c_void_p(page_table.data_ptr()), ctypes.POINTER(ctypes.c_int32)),
+        ctypes.byref(wf.c), int(generation) & 0xFFFFFFFF, _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_kv_append_publish_fp8")
+
+
+def kv_dequant_published(k_codes, v_codes, k_scale, v_scale, k_pool, v_pool, layer: int,
+                         chunk: int, page_table, wf: WavefrontDesc, flags_row, generation: int,
+                         stream=None) -> None:
+    """wf_kv_dequant_published: kv_dequant that first waits for ``flags_row[chunk]`` (device
+    uint32 [WF_MAX_CHUNKS]) to reach ``generation``."""
+    geo = _fp8_pool_shape(k_codes, v_codes, k_scale, v_scale)
+    if _pool_shape(k_pool, v_pool) != geo:
+        raise ValueError(f"bf16 pool {tuple(k_pool.shape)} differs from the FP8 pool {geo}")
+    _check_page_table(page_table, layer, wf)
+    if flags_row.numel() < len(wf.chunk_offsets) - 1:
+        raise ValueError(f"flags_row: needs >= {len(wf.chunk_offsets) - 1} words")
+    for t, n, d in ((k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
+                    (page_table, "page_table", "i32"), (flags_row, "flags_row", "u32")):
+        _check_tensor(t, n, d)
+    src = _fp8_pool_struct(k_codes, v_codes, k_scale, v_scale)
+    dst = _pool_struct(k_pool, v_pool)
+    rc = lib.wf_kv_dequant_published(ctypes.byref(src), ctypes.byref(dst), int(layer),
+                                     int(chunk),
+                                     ctypes.cast(ctypes.c_void_p(page_table.data_ptr()),
+                                                 ctypes.POINTER(ctypes.c_int32)),
+                                     ctypes.byref(wf.c), flags_row.data_ptr(),
+                                     int(generation) & 0xFFFFFFFF, _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_kv_dequant_published")
 
 
 def attn_forward(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: float, out,

@@ -20,7 +20,6 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libwf_b200.so")
 SOURCES = [os.path.join(CSRC, "wf_api.cu"), os.path.join(CSRC, "wf_window.cpp")]
 DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "attn_kernel.cuh",
-                                                      "attn_pair_kernel.cuh",
                                                       "append_kernel.cuh", "combine_kernel.cuh",
                                                       "fp8_kernel.cuh",
                                                       "publish_kernel.cuh")] + \

@@ -29,9 +29,14 @@
 // Issue order: S_0(0), S_1(0), then for every tile j: P.V_0(j), S_0(j+1), P.V_1(j), S_1(j+1).
 // The two Q tiles run half a period apart: while the softmax of one tile computes P, the tensor
 // pipe works on the other tile's P.V and QK^T, and the two softmax warpgroups do not compete for
-// the exp unit at the same time.  S_q(j+1) overwrites the columns P.V_q(j) reads P from; PTX
-// orders consecutive MMAs only for the same accumulator, so S_q(j+1) is issued after o_done[q]
-// reports that P.V_q(j) completed.
+// the exp unit at the same time.  S_q(j+1) overwrites the columns P.V_q(j) reads P from, and is
+// issued right behind it by the same thread without waiting for P.V_q(j) to complete: the tensor
+// core executes one thread's MMAs in issue order, so P.V_q(j) has read its A operand before
+// S_q(j+1) writes those columns.  PTX lists same-accumulator MMA pairs among its pipelined
+// (ordered) pairs; this different-accumulator order is the one NVIDIA's own CUTLASS Blackwell
+// attention mainloop relies on in the same situation (QK^T into S issued straight after the P.V
+// that reads P from S's columns).  Waiting for completion instead cost 4.5 % on the 1.3B 5-step
+// wavefront.
 //
 // Synchronisation (all mbarriers, all waits bounded):
 //   q_full          TMA -> MMA          Q tiles landed
@@ -39,7 +44,8 @@
 //   kv_empty[s]     MMA commit -> TMA   slot s free again (both Q tiles' MMAs on it completed)
 //   s_full[q]       MMA commit -> softmax q   S_q of the current tile ready
 //   p_full[q]       softmax q -> MMA    P_q written to TMEM (and O_q rescaled if needed)
-//   o_done[q]       MMA commit -> MMA / softmax   P.V_q of the current tile completed
+//   o_done[q]       MMA commit -> softmax q   P.V_q of the current tile completed (O rescale,
+//                                             epilogue)
 //   v_zeroed        TMA warp -> MMA     tail rows of the last V tile zeroed
 #pragma once
 
@@ -70,10 +76,6 @@ static_assert(kRegSoftmax % 8 == 0 && kRegOther % 8 == 0 && kRegOther >= 24,
               "setmaxnreg counts are multiples of 8");
 static_assert(2 * 128 * kRegSoftmax + 128 * kRegOther <= 384 * 168, "split exceeds the launch");
 constexpr int kMaxQChunks = 64;
-#ifndef WF_PT_CACHE
-#define WF_PT_CACHE 0      // 0: each tile reads its page-table entries from global memory
-#endif
-constexpr int kPtCache = WF_PT_CACHE;   // page-table entries a producer keeps in shared memory
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;   // 0.2 s when draining
 
@@ -88,7 +90,6 @@ struct AttnParams {
   unsigned* grid_abort;
   int T_q, H, num_pages, page_size, total_rows, box_rows, n_pairs;
   int head_group;     // heads per group of the dispatch order (divides H)
-  int box_rows_v;     // V box rows (CTA-pair kernel: V half-tiles of 128 keys)
   float sl2;  // scale * log2(e)
   unsigned launch_id;
   int nqc;                          // non-empty query chunks
@@ -114,24 +115,11 @@ __device__ __forceinline__ int kv_end_of_row(const AttnParams& p, int r) {
   return p.qc_kv_end[p.nqc - 1];
 }
 
-// The producer warp copies the page-table entries of the unit's key range into shared memory
-// once (up to kPtCache of them), so each K/V tile costs a shared-memory read instead of a
-// dependent global load.  Returns the number of cached entries.
-__device__ __forceinline__ int cache_page_table(const AttnParams& p, int* pt_s, int n_max,
-                                                int lane) {
-  const int pages = (n_max + p.page_size - 1) / p.page_size;
-  const int n = min(pages, kPtCache);
-  for (int i = lane; i < n; i += 32) pt_s[i] = __ldg(p.page_table + i);
-  __syncwarp();
-  return n;
-}
-
 // Physical pool row of logical token `tok` (< n_max); entries outside the pool are recorded
 // as WF_ERR_PAGE_OOB and read as page 0.
-__device__ __forceinline__ int pool_row(const AttnParams& p, const int* pt_s, int n_cached,
-                                        int tok) {
+__device__ __forceinline__ int pool_row(const AttnParams& p, int tok) {
   const int idx = tok / p.page_size;
-  int pg = idx < n_cached ? pt_s[idx] : __ldg(p.page_table + idx);
+  int pg = __ldg(p.page_table + idx);
   if (pg < 0 || pg >= p.num_pages) {
     atomicCAS(p.status, 0, 5 /* WF_ERR_PAGE_OOB */);
     pg = 0;
@@ -164,8 +152,7 @@ struct AttnSmem {
   static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NS, B_S = 1 + 2 * NS,
                        B_P = B_S + kNQT, B_O = B_P + kNQT, B_DRAIN = B_O + kNQT,
                        B_VZ = B_DRAIN + 1, NBAR = B_VZ + 1;
-  static constexpr uint32_t PT_OFF = BAR_OFF + NBAR * 8;   // page-table cache
-  static constexpr uint32_t MISC_OFF = PT_OFF + kPtCache * 4;
+  static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr uint32_t BYTES = MISC_OFF + 16;
   static constexpr uint32_t ALLOC = BYTES + 1024;        // slack for 1024-byte alignment
   static_assert(ALLOC <= 227u * 1024u, "shared memory per CTA exceeds 227 KB");
@@ -304,7 +291,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // no visible key yet (possible in a later key split): every p is exactly 0
         const float mref = m2 == -INFINITY ? 0.f : m2;
         const float2 negm = make_float2(-mref, -mref);
-        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        // The row sum l adds the weights as P.V uses them -- rounded to bf16 -- so O / l is a
+        // convex combination of the visible values (V = 1 gives exactly 1).
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[BN / 2];
         if (!masked) {
   #pragma unroll
@@ -317,23 +306,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               e.x = ex2_approx(x.x);
               e.y = ex2_approx(x.y);
             }
-            if (i & 1) acc1 = __fadd2_rn(acc1, e); else acc0 = __fadd2_rn(acc0, e);
             pk[i] = pack_bf16x2(e.x, e.y);
+            acc[i & 3] = add_bf16x2(acc[i & 3], pk[i]);
           }
         } else {
   #pragma unroll
           for (int i = 0; i < BN / 2; ++i) {
             const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2x2, negm);
-            const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            if (i & 1) acc1 = __fadd2_rn(acc1, e); else acc0 = __fadd2_rn(acc0, e);
-            pk[i] = pack_bf16x2(e.x, e.y);
+            pk[i] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
+            acc[i & 3] = add_bf16x2(acc[i & 3], pk[i]);
           }
         }
   #pragma unroll
         for (int h = 0; h < BN / 64; ++h)
           tmem_st32(tS + 32u * h, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h]));
-        const float2 acc = __fadd2_rn(acc0, acc1);
-        l += acc.x + acc.y;
+        l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(L::B_P + q));
@@ -404,12 +391,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         m0 + qt * kBM, bar(L::B_Q));
       }
       // Physical row of box b of tile t (past the pool -- TMA fills zeros -- beyond n_max).
-      int* const pt_s = reinterpret_cast<int*>(base_ptr + L::PT_OFF);
-      const int n_cached = cache_page_table(p, pt_s, n_max, lane);
       auto box_row = [&](int t, int b) -> int {
         const int tok = (kb + t) * BN + b * R;
         if (b >= nb || t >= nk || tok >= n_max) return p.total_rows;
-        return pool_row(p, pt_s, n_cached, tok);
+        return pool_row(p, tok);
       };
       int ready = 0;                                        // chunks known to be published
       for (int j = 0; j < nk && ok; ++j) {
@@ -535,10 +520,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (q == kNQT - 1) umma_commit(bar(L::B_KVE + slotv));   // V_j free
           if (j + 1 < nk) {
             if (q == 0) ok = wait_k(j + 1);
-            if (ok) ok = mbar_wait(bar(L::B_O + q), j & 1, w);      // P.V_q(j) done reading P
             if (!ok) break;
-            tc_fence_after();
-            issue_s_q(j + 1, q);
+            issue_s_q(j + 1, q);            // in issue order behind P.V_q(j), see the header
             if (q == kNQT - 1) umma_commit(bar(L::B_KVE + (2 * (j + 1)) % NS));   // K_{j+1} free
           }
         }

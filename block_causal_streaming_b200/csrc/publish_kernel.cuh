@@ -80,13 +80,25 @@ __global__ void __launch_bounds__(kPublishThreads)
   }
 }
 
-// Runs after wf_publish_kernel on the same stream, so every row is written; thread d makes them
-// visible system-wide and then releases destination d's flag.
+// Runs after wf_publish_kernel on the same stream, so every row is written; lane d makes them
+// visible system-wide and then releases destination d's flag.  A row whose page-table entry is
+// outside the pool was skipped by wf_publish_kernel (and recorded as WF_ERR_PAGE_OOB on this
+// device), so the chunk is incomplete: its flag is then raised in no pool, and a consumer waits
+// (and at worst times out) rather than reading stale pages as if they were the new chunk.
 __global__ void wf_publish_flags_kernel(const __grid_constant__ PublishParams p) {
-  const int d = threadIdx.x;
-  if (d >= p.n_dst || p.dst[d].flag == nullptr) return;
+  const int lane = threadIdx.x;
+  bool bad = false;
+  if (p.rows > 0) {
+    const int first = p.token0 / p.page_size, last = (p.token0 + p.rows - 1) / p.page_size;
+    for (int i = first + lane; i <= last; i += 32) {
+      const int pg = __ldg(p.pt_row + i);
+      bad = bad || pg < 0 || pg >= p.num_pages;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad)) return;
+  if (lane >= p.n_dst || p.dst[lane].flag == nullptr) return;
   __threadfence_system();
-  asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p.dst[d].flag), "r"(p.generation)
+  asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p.dst[lane].flag), "r"(p.generation)
                : "memory");
 }
 

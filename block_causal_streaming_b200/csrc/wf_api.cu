@@ -14,7 +14,6 @@
 #include "../../include/wf.h"
 #include "append_kernel.cuh"
 #include "attn_kernel.cuh"
-#include "attn_pair_kernel.cuh"
 #include "combine_kernel.cuh"
 #include "fp8_kernel.cuh"
 #include "publish_kernel.cuh"
@@ -25,10 +24,6 @@ __device__ int g_wf_status = 0;
 // Launch id of the last attention launch in which a bounded wait ran out; every other CTA of
 // that launch stops as soon as it sees it.
 __device__ unsigned g_wf_abort = 0;
-
-#ifndef WF_ATTN_PAIR
-#define WF_ATTN_PAIR 0
-#endif
 
 // Scratch of wf_attn_forward_split_noalloc: one static array per device, so that entry point
 // needs no allocation.  96 MiB holds the partial results of 3 key splits of a 4680-row, 12-head,
@@ -42,7 +37,8 @@ constexpr int kMaxDevices = 64;
 std::atomic<unsigned> g_launch_counter{1};
 
 struct DeviceState {
-  bool ready = false;
+  // Set (release) once the fields below are filled; read (acquire) without the lock.
+  std::atomic<bool> ready{false};
   bool sm100 = false;
   int* status = nullptr;
   unsigned* abort_word = nullptr;
@@ -60,9 +56,9 @@ int device_state(DeviceState** out) {
     return WF_ERR_NO_DEVICE;
   }
   DeviceState& d = g_dev[dev];
-  if (!d.ready) {
+  if (!d.ready.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lock(g_dev_mu);
-    if (!d.ready) {
+    if (!d.ready.load(std::memory_order_relaxed)) {
       cudaDeviceProp prop;
       if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
         cudaGetLastError();
@@ -85,15 +81,12 @@ int device_state(DeviceState** out) {
                                  wfk::AttnSmem<128>::ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<64, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 wfk::AttnSmem<64>::ALLOC) != cudaSuccess ||
-            cudaFuncSetAttribute(wfk::wf_attn_pair_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 wfk::PairSmem::ALLOC) != cudaSuccess) {
+                                 wfk::AttnSmem<64>::ALLOC) != cudaSuccess) {
           cudaGetLastError();
           return WF_ERR_CUDA;
         }
       }
-      d.ready = true;
+      d.ready.store(true, std::memory_order_release);
     }
   }
   if (!d.sm100) return WF_ERR_NO_DEVICE;
@@ -317,7 +310,6 @@ struct AttnLaunch {
   QueryPlan qp;
   DeviceState* d = nullptr;
   int D = 0;
-  bool use_pair = false;
   float* lse_out = nullptr;   // the caller's lse (written by the combine pass when split)
 };
 
@@ -346,18 +338,15 @@ int prepare_attention(const void* q, const wf_kv_pool_t* kv_pages, const int32_t
   const int H = kv_pages->num_heads, D = kv_pages->head_dim, ps = kv_pages->page_size;
   static_assert(alignof(wfk::AttnParams) >= 64, "tensor maps need 64-byte alignment");
   L->D = D;
-  // CTA pairs run head_dim 128; a box never crosses a page or a tile edge
-  L->use_pair = (D == 128) && WF_ATTN_PAIR;
-  const int box_rows = gcd_int(ps, L->use_pair ? 64 : wfk::kBN);
-  const int box_rows_v = gcd_int(ps, L->use_pair ? wfk::kPairBN : wfk::kBN);
+  // a box never crosses a page or a tile edge
+  const int box_rows = gcd_int(ps, wfk::kBN);
   const int64_t total_rows = static_cast<int64_t>(kv_pages->num_pages) * ps;
   if (!encode_rows(&p.tm_q, q, D, H, t_q, wfk::kBM, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
       !encode_rows(&p.tm_k, kv_pages->k_pool, D, H, total_rows, box_rows,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
-      !encode_rows(&p.tm_v, kv_pages->v_pool, D, H, total_rows, box_rows_v,
+      !encode_rows(&p.tm_v, kv_pages->v_pool, D, H, total_rows, box_rows,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
     return WF_ERR_CUDA;
-  p.box_rows_v = box_rows_v;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse_or_null;
   L->lse_out = lse_or_null;
@@ -399,9 +388,7 @@ int launch_attention(AttnLaunch* L, cudaStream_t s) {
   const int64_t grid = static_cast<int64_t>(p.n_pairs) * p.H * p.n_splits;
   const unsigned g = static_cast<unsigned>(grid);
   const bool wait = p.flags != nullptr;
-  if (L->use_pair)
-    wfk::wf_attn_pair_kernel<<<2 * g, wfk::kPairThreads, wfk::PairSmem::ALLOC, s>>>(p);
-  else if (L->D == 128 && !wait)
+  if (L->D == 128 && !wait)
     wfk::wf_attn_fwd_kernel<128><<<g, wfk::kAttnThreads, wfk::AttnSmem<128>::ALLOC, s>>>(p);
   else if (L->D == 128)
     wfk::wf_attn_fwd_kernel<128, true><<<g, wfk::kAttnThreads, wfk::AttnSmem<128>::ALLOC, s>>>(
@@ -527,7 +514,6 @@ int wf_attn_forward_split(const void* q, const wf_kv_pool_t* kv_pages,
   if (rc || L.p.T_q == 0) return rc;
   int S = splits > 0 ? splits : choose_splits(L.qp, L.p.H, L.d->num_sms);
   S = std::min(S, max_splits(L.qp));
-  if (L.use_pair) S = 1;                       // the CTA-pair kernel has no key splits
   if (S > 1) {
     const size_t need = split_workspace_bytes(L.qp, L.p.H, L.D, S);
     if (workspace == nullptr || !aligned16(workspace)) return WF_ERR_INVALID_ARG;
@@ -547,7 +533,6 @@ int wf_attn_forward_split_noalloc(const void* q, const wf_kv_pool_t* kv_pages,
   if (rc || L.p.T_q == 0) return rc;
   int S = splits > 0 ? splits : choose_splits(L.qp, L.p.H, L.d->num_sms);
   S = std::min(S, max_splits(L.qp));
-  if (L.use_pair) S = 1;
   if (S > 1) {
     if (split_workspace_bytes(L.qp, L.p.H, L.D, S) > kScratchBytes) return WF_ERR_CAPACITY;
     void* scratch = nullptr;
@@ -624,7 +609,6 @@ int wf_attn_forward_published(const void* q, const wf_kv_pool_t* kv_pages,
   AttnLaunch L;
   const int rc = prepare_attention(q, kv_pages, page_table_row, wf, scale, out, lse_or_null, &L);
   if (rc || L.p.T_q == 0) return rc;
-  if (L.use_pair) return WF_ERR_SHAPE;         // the CTA-pair kernel has no publication wait
   int S = splits > 0 ? splits : choose_splits(L.qp, L.p.H, L.d->num_sms);
   S = std::min(S, max_splits(L.qp));
   if (S > 1) {
@@ -723,8 +707,9 @@ int fp8_chunk_args(const wf_kv_pool_fp8_t* pool, int layer, int chunk, const int
   return WF_OK;
 }
 
-int fp8_blocks(const DeviceState* d, int rows, int heads) {
-  const int64_t warps = static_cast<int64_t>(rows) * heads;
+// One warp per token.
+int fp8_blocks(const DeviceState* d, int rows) {
+  const int64_t warps = rows;
   const int per_block = wfk::kFp8Threads / 32;
   int64_t blocks = (warps + per_block - 1) / per_block;
   const int64_t cap = static_cast<int64_t>(d->num_sms) * 8;   // 64 warps per SM in flight
@@ -733,32 +718,144 @@ int fp8_blocks(const DeviceState* d, int rows, int heads) {
 
 }  // namespace
 
+}  // extern "C"
+
+namespace {
+
+// Quantize one chunk into pool and the FP8 peers (shared by the append and the publication).
+int launch_quant(const wf_kv_pool_fp8_t* pool, const wf_fp8_dst_t* peers, int num_peers,
+                 int t0, int rows, const int32_t* row, const void* k, const void* v,
+                 cudaStream_t s) {
+  DeviceState* d = nullptr;
+  const int rc = device_state(&d);
+  if (rc) return rc;
+  wfk::QuantParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.pt_row = row;
+  p.status = d->status;
+  p.token0 = t0;
+  p.rows = rows;
+  p.H = pool->num_heads;
+  p.page_size = pool->page_size;
+  p.num_pages = pool->num_pages;
+  p.n_dst = 1 + num_peers;
+  p.dst[0] = {static_cast<uint8_t*>(pool->k_codes), static_cast<uint8_t*>(pool->v_codes),
+              pool->k_scale, pool->v_scale};
+  for (int i = 0; i < num_peers; ++i)
+    p.dst[1 + i] = {static_cast<uint8_t*>(peers[i].k_codes),
+                    static_cast<uint8_t*>(peers[i].v_codes), peers[i].k_scale, peers[i].v_scale};
+  const int blocks = fp8_blocks(d, rows);
+  if (pool->head_dim == 128)
+    wfk::wf_quant_append_kernel<128><<<blocks, wfk::kFp8Threads, 0, s>>>(p);
+  else
+    wfk::wf_quant_append_kernel<64><<<blocks, wfk::kFp8Threads, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+// Dequantize one chunk; with flag != null every block first waits for it to reach `generation`.
+int launch_dequant(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int t0, int rows,
+                   const int32_t* row, const uint32_t* flag, uint32_t generation,
+                   cudaStream_t s) {
+  DeviceState* d = nullptr;
+  const int rc = device_state(&d);
+  if (rc) return rc;
+  wfk::DequantParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.k_codes = static_cast<const uint8_t*>(src->k_codes);
+  p.v_codes = static_cast<const uint8_t*>(src->v_codes);
+  p.k_scale = src->k_scale;
+  p.v_scale = src->v_scale;
+  p.k_pool = static_cast<__nv_bfloat16*>(dst->k_pool);
+  p.v_pool = static_cast<__nv_bfloat16*>(dst->v_pool);
+  p.pt_row = row;
+  p.status = d->status;
+  p.token0 = t0;
+  p.rows = rows;
+  p.H = src->num_heads;
+  p.page_size = src->page_size;
+  p.num_pages = src->num_pages;
+  p.flag = flag;
+  p.generation = generation;
+  p.grid_abort = d->abort_word;
+  p.launch_id = g_launch_counter.fetch_add(1);
+  if (p.launch_id == 0) p.launch_id = g_launch_counter.fetch_add(1);
+  const int blocks = fp8_blocks(d, rows);
+  const bool wait = flag != nullptr;
+  if (src->head_dim == 128 && !wait)
+    wfk::wf_dequant_kernel<128, false><<<blocks, wfk::kFp8Threads, 0, s>>>(p);
+  else if (src->head_dim == 128)
+    wfk::wf_dequant_kernel<128, true><<<blocks, wfk::kFp8Threads, 0, s>>>(p);
+  else if (!wait)
+    wfk::wf_dequant_kernel<64, false><<<blocks, wfk::kFp8Threads, 0, s>>>(p);
+  else
+    wfk::wf_dequant_kernel<64, true><<<blocks, wfk::kFp8Threads, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int same_geometry(const wf_kv_pool_fp8_t* a, const wf_kv_pool_t* b) {
+  return b->num_pages == a->num_pages && b->page_size == a->page_size &&
+         b->num_heads == a->num_heads && b->head_dim == a->head_dim;
+}
+
+}  // namespace
+
+extern "C" {
+
 int wf_kv_append_fp8(const wf_kv_pool_fp8_t* pool, int layer, int chunk, const void* k,
                      const void* v, const int32_t* page_table, const wf_wavefront_t* wf,
                      wf_stream_t stream) {
   int t0 = 0, rows = 0;
   const int32_t* row = nullptr;
-  int rc = fp8_chunk_args(pool, layer, chunk, page_table, wf, &t0, &rows, &row);
+  const int rc = fp8_chunk_args(pool, layer, chunk, page_table, wf, &t0, &rows, &row);
   if (rc) return rc;
   if (rows == 0) return WF_OK;
   if (k == nullptr || v == nullptr || !aligned16(k) || !aligned16(v)) return WF_ERR_INVALID_ARG;
-  DeviceState* d = nullptr;
-  rc = device_state(&d);
+  return launch_quant(pool, nullptr, 0, t0, rows, row, k, v,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int wf_kv_append_publish_fp8(const wf_kv_pool_fp8_t* pool, uint32_t* flags,
+                             const wf_fp8_dst_t* peers, int num_peers, int layer, int chunk,
+                             const void* k, const void* v, const int32_t* page_table,
+                             const wf_wavefront_t* wf, uint32_t generation, wf_stream_t stream) {
+  int t0 = 0, rows = 0;
+  const int32_t* row = nullptr;
+  int rc = fp8_chunk_args(pool, layer, chunk, page_table, wf, &t0, &rows, &row);
   if (rc) return rc;
-  const int blocks = fp8_blocks(d, rows, pool->num_heads);
+  if (num_peers < 0 || num_peers > wfk::kMaxFp8Dst - 1 || (num_peers > 0 && peers == nullptr))
+    return WF_ERR_INVALID_ARG;
+  for (int i = 0; i < num_peers; ++i)
+    if (peers[i].k_codes == nullptr || peers[i].v_codes == nullptr ||
+        peers[i].k_scale == nullptr || peers[i].v_scale == nullptr ||
+        !aligned16(peers[i].k_codes) || !aligned16(peers[i].v_codes) ||
+        !aligned16(peers[i].k_scale) || !aligned16(peers[i].v_scale) ||
+        (reinterpret_cast<uintptr_t>(peers[i].flags) & 3u))
+      return WF_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(flags) & 3u) return WF_ERR_INVALID_ARG;
+  if (rows > 0 && (k == nullptr || v == nullptr || !aligned16(k) || !aligned16(v)))
+    return WF_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  auto ks = static_cast<const __nv_bfloat16*>(k);
-  auto vs = static_cast<const __nv_bfloat16*>(v);
-  auto kc = static_cast<uint8_t*>(pool->k_codes);
-  auto vc = static_cast<uint8_t*>(pool->v_codes);
-  if (pool->head_dim == 128)
-    wfk::wf_quant_append_kernel<128><<<blocks, wfk::kFp8Threads, 0, s>>>(
-        ks, vs, kc, vc, pool->k_scale, pool->v_scale, row, t0, rows, pool->num_heads,
-        pool->page_size, pool->num_pages, d->status);
-  else
-    wfk::wf_quant_append_kernel<64><<<blocks, wfk::kFp8Threads, 0, s>>>(
-        ks, vs, kc, vc, pool->k_scale, pool->v_scale, row, t0, rows, pool->num_heads,
-        pool->page_size, pool->num_pages, d->status);
+  if (rows > 0) {
+    rc = launch_quant(pool, peers, num_peers, t0, rows, row, k, v, s);
+    if (rc) return rc;
+  }
+  // the generation flags, released once every row is written (the kernel of the bf16 path)
+  wfk::PublishParams fp;
+  std::memset(&fp, 0, sizeof(fp));
+  fp.pt_row = row;
+  fp.token0 = t0;
+  fp.rows = rows;
+  fp.page_size = pool->page_size;
+  fp.num_pages = pool->num_pages;
+  fp.generation = generation;
+  const size_t flag_at = static_cast<size_t>(layer) * WF_MAX_CHUNKS + chunk;
+  fp.n_dst = 1 + num_peers;
+  fp.dst[0].flag = flags != nullptr ? flags + flag_at : nullptr;
+  for (int i = 0; i < num_peers; ++i)
+    fp.dst[1 + i].flag = peers[i].flags != nullptr ? peers[i].flags + flag_at : nullptr;
+  wfk::wf_publish_flags_kernel<<<1, 32, 0, s>>>(fp);
   return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
@@ -770,28 +867,27 @@ int wf_kv_dequant(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int laye
   if (rc) return rc;
   rc = validate_pool(dst);
   if (rc) return rc;
-  if (dst->num_pages != src->num_pages || dst->page_size != src->page_size ||
-      dst->num_heads != src->num_heads || dst->head_dim != src->head_dim)
-    return WF_ERR_SHAPE;
+  if (!same_geometry(src, dst)) return WF_ERR_SHAPE;
   if (rows == 0) return WF_OK;
-  DeviceState* d = nullptr;
-  rc = device_state(&d);
+  return launch_dequant(src, dst, t0, rows, row, nullptr, 0,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int wf_kv_dequant_published(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int layer,
+                            int chunk, const int32_t* page_table, const wf_wavefront_t* wf,
+                            const uint32_t* flags_row, uint32_t generation, wf_stream_t stream) {
+  int t0 = 0, rows = 0;
+  const int32_t* row = nullptr;
+  int rc = fp8_chunk_args(src, layer, chunk, page_table, wf, &t0, &rows, &row);
   if (rc) return rc;
-  const int blocks = fp8_blocks(d, rows, src->num_heads);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  auto kc = static_cast<const uint8_t*>(src->k_codes);
-  auto vc = static_cast<const uint8_t*>(src->v_codes);
-  auto kp = static_cast<__nv_bfloat16*>(dst->k_pool);
-  auto vp = static_cast<__nv_bfloat16*>(dst->v_pool);
-  if (src->head_dim == 128)
-    wfk::wf_dequant_kernel<128><<<blocks, wfk::kFp8Threads, 0, s>>>(
-        kc, vc, src->k_scale, src->v_scale, kp, vp, row, t0, rows, src->num_heads,
-        src->page_size, src->num_pages, d->status);
-  else
-    wfk::wf_dequant_kernel<64><<<blocks, wfk::kFp8Threads, 0, s>>>(
-        kc, vc, src->k_scale, src->v_scale, kp, vp, row, t0, rows, src->num_heads,
-        src->page_size, src->num_pages, d->status);
-  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+  rc = validate_pool(dst);
+  if (rc) return rc;
+  if (!same_geometry(src, dst)) return WF_ERR_SHAPE;
+  if (flags_row == nullptr || (reinterpret_cast<uintptr_t>(flags_row) & 3u))
+    return WF_ERR_INVALID_ARG;
+  if (rows == 0) return WF_OK;
+  return launch_dequant(src, dst, t0, rows, row, flags_row + chunk, generation,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 int wf_selftest_timeout(unsigned timeout_us, wf_stream_t stream) {

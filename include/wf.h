@@ -215,8 +215,7 @@ int wf_kv_append_publish(const wf_kv_pool_t* pool, uint32_t* flags, const wf_poo
  * flags_row: device uint32 [WF_MAX_CHUNKS], this layer's row of this GPU's flag array; every
  * chunk the queries see (own chunk included) must be flagged, e.g. by wf_kv_append_publish.
  * A wait that lasts longer than 2 s stops the kernel and records WF_ERR_TIMEOUT (read with
- * wf_check_status).  Other arguments and errors as wf_attn_forward_split; WF_ERR_SHAPE if the
- * library was built with the CTA-pair kernel.
+ * wf_check_status).  Other arguments and errors as wf_attn_forward_split.
  */
 int wf_attn_forward_published(const void* q, const wf_kv_pool_t* kv_pages,
                               const int32_t* page_table_row, const wf_wavefront_t* wf,
@@ -261,7 +260,9 @@ typedef struct {
  * wf_kv_append_fp8 -- wf_kv_append into an FP8 pool.  Each (token, head) row x of head_dim values,
  * with amax its largest magnitude, is stored as scale = amax / 448 and codes
  * e4m3(x * (448 / amax)), rounded to nearest even and saturated at +-448; both divisions and
- * the product are fp32 round-to-nearest.  A row of zeros stores scale 0 and zero codes.
+ * the product are fp32 round-to-nearest.  A row of zeros stores scale 0 and zero codes, and so
+ * does a row whose 448 / amax overflows fp32 (amax below about 1.3e-36); their codes keep the
+ * values' signs.
  * Arguments and errors as wf_kv_append (k, v: device bf16 [L_c][H][D], 16-byte aligned).
  */
 int wf_kv_append_fp8(const wf_kv_pool_fp8_t* pool, int layer, int chunk, const void* k,
@@ -276,6 +277,46 @@ int wf_kv_append_fp8(const wf_kv_pool_fp8_t* pool, int layer, int chunk, const v
  */
 int wf_kv_dequant(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int layer, int chunk,
                   const int32_t* page_table, const wf_wavefront_t* wf, wf_stream_t stream);
+
+/*
+ * FP8 publication (project page, "03 End-to-end KV transport", items 01 "Precision" and 03
+ * "Layout": the producer sends each chunk's K/V in FP8 straight into the consumers' buffers,
+ * which convert them back before attention).  The transport moves head_dim + 4 bytes per
+ * (token, head) row of each tensor instead of 2 head_dim (0.516 x at head_dim 128).
+ */
+typedef struct {
+  void* k_codes;       /* the destination GPU's FP8 pool, same geometry as the source */
+  void* v_codes;
+  float* k_scale;
+  float* v_scale;
+  uint32_t* flags;     /* that GPU's flag array [num_layers][WF_MAX_CHUNKS], or NULL */
+} wf_fp8_dst_t;
+
+/*
+ * wf_kv_append_publish_fp8 -- wf_kv_append_fp8 into `pool` and, in the same kernel (the bf16
+ * chunk is read and quantized once), into every peer's FP8 pool (up to 8, plain stores through
+ * peer pointers), then raises word (layer, chunk) of `flags` (may be NULL) and of every peer's
+ * flags to `generation` as wf_kv_append_publish does: after a system-wide fence, with a
+ * system-scope release, and not at all when a row of the chunk has a page outside the pool
+ * (WF_ERR_PAGE_OOB is then recorded).  Errors as wf_kv_append_fp8; WF_ERR_INVALID_ARG for more
+ * than 8 peers or a null/misaligned peer pointer.  Asynchronous on `stream`.
+ */
+int wf_kv_append_publish_fp8(const wf_kv_pool_fp8_t* pool, uint32_t* flags,
+                             const wf_fp8_dst_t* peers, int num_peers, int layer, int chunk,
+                             const void* k, const void* v, const int32_t* page_table,
+                             const wf_wavefront_t* wf, uint32_t generation, wf_stream_t stream);
+
+/*
+ * wf_kv_dequant_published -- wf_kv_dequant of a chunk another GPU publishes into `src`: every
+ * block first waits until flags_row[chunk] has reached `generation` (signed 32-bit difference
+ * >= 0, system-scope acquire), then converts.  flags_row: device uint32 [WF_MAX_CHUNKS], this
+ * layer's row of this GPU's flag array.  A wait longer than 2 s records WF_ERR_TIMEOUT (read with
+ * wf_check_status) and writes nothing.  A plain wf_attn_forward on `dst`, later on the same
+ * stream, then reads the chunk.  Other arguments and errors as wf_kv_dequant.
+ */
+int wf_kv_dequant_published(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int layer,
+                            int chunk, const int32_t* page_table, const wf_wavefront_t* wf,
+                            const uint32_t* flags_row, uint32_t generation, wf_stream_t stream);
 
 /*
  * Rolling context window: the plan of one round of a stream (host only, no device work).

@@ -13,7 +13,9 @@ readings taken here:
   page, so a per-page scale could not be fixed when the first of them is written.  For a row with
   largest magnitude ``amax > 0``: ``inv = 448 / amax`` and ``scale = amax / 448``, both fp32
   divisions, and ``code = e4m3(x * inv)`` with an fp32 product.  A row of zeros gets scale 0 and
-  codes 0.  Every step is fp32, as on the device, because these values decide the integer codes.
+  codes 0, and so does a row whose ``448 / amax`` overflows fp32 (``amax`` below about 1.3e-36):
+  no scale could carry it back, and values that small mean nothing in bf16 K/V.  Every step is
+  fp32, as on the device, because these values decide the integer codes.
 * **Dequantization:** ``bf16_rne(fp32(decode(code)) * scale)``, which is what attention reads.
 
 Every function is pinned by ``tests/test_oracle_fp8.py``: the value table against the format's
@@ -70,8 +72,12 @@ def quantize_rows(x) -> tuple:
     amax = np.max(np.abs(x), axis=-1).astype(np.float32)
     nz = amax > 0
     safe = np.where(nz, amax, np.float32(1)).astype(np.float32)
-    inv = np.where(nz, np.float32(E4M3_MAX) / safe, np.float32(0)).astype(np.float32)
-    scale = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(0)).astype(np.float32)
+    with np.errstate(over="ignore"):
+        inv = (np.float32(E4M3_MAX) / safe).astype(np.float32)
+    # a row of zeros, or one so small that 448 / amax overflows fp32, is stored as zeros
+    live = nz & np.isfinite(inv)
+    inv = np.where(live, inv, np.float32(0)).astype(np.float32)
+    scale = np.where(live, safe / np.float32(E4M3_MAX), np.float32(0)).astype(np.float32)
     y = (x * inv[..., None]).astype(np.float32)
     return e4m3_encode(y), scale
 

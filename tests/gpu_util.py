@@ -69,3 +69,33 @@ def sample_rows(wl: Workload, per_chunk: int = 3, seed: int = 0):
     heads = [int(h) for h in rng.integers(0, wl.heads, size=len(rows))]
     heads[0], heads[-1] = 0, wl.heads - 1
     return rows, heads
+
+
+UNIT_ROWS = 256   # query rows of one attention work unit (two 128-row Q tiles)
+
+
+def whole_units(wl: Workload, seed: int = 0, interior: bool = True):
+    """Every head of every row of whole 256-row work units: for each query chunk the unit that
+    holds its first row and the one that holds its last row (these straddle chunk boundaries
+    unless a boundary falls on a unit edge) and, with `interior`, one interior unit drawn at
+    random; the last unit of the wavefront, whose rows see the most keys, is always among them.
+    Returns
+    (rows, heads, units), rows/heads flattened so that pair i is (rows[i], heads[i])."""
+    rng = np.random.default_rng(seed)
+    off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
+    t_ctx, t_q = off[nctx], wl.t_q
+    units = {(t_q - 1) // UNIT_ROWS}
+    for c in range(nctx, wl.num_chunks):
+        a, b = off[c] - t_ctx, off[c + 1] - t_ctx
+        if b <= a:
+            continue
+        first, last = a // UNIT_ROWS, (b - 1) // UNIT_ROWS
+        units.update({first, last})
+        if interior and last - first > 1:
+            units.add(int(rng.integers(first + 1, last)))
+    units = sorted(units)
+    rows = np.concatenate([np.arange(u * UNIT_ROWS, min((u + 1) * UNIT_ROWS, t_q))
+                           for u in units]).astype(np.int32)
+    heads = np.tile(np.arange(wl.heads, dtype=np.int32), len(rows))
+    rows = np.repeat(rows, wl.heads)
+    return rows, heads, units

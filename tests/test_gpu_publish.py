@@ -13,7 +13,8 @@ import pytest
 import torch
 
 import oracle
-from block_causal_streaming_b200 import (WF_ERR_TIMEOUT, WF_OK, attn_forward_published,
+from block_causal_streaming_b200 import (WF_ERR_PAGE_OOB, WF_ERR_TIMEOUT, WF_OK,
+                                         attn_forward_published,
                                          attn_workspace_size, check_status, kv_append_publish)
 from block_causal_streaming_b200.layer import PagedPool
 from block_causal_streaming_b200.wave import new_flags
@@ -158,3 +159,24 @@ def test_publication_at_head_dim_64_with_splits():
         out = P.attend(i, splits=2)
         assert check_status() == WF_OK
         assert_parity(out.float().cpu().numpy(), ref, f"pool {i}")
+
+
+def test_a_chunk_with_a_page_outside_the_pool_is_not_published():
+    """A page-table entry outside the pool makes the writer skip those rows; the chunk is then
+    incomplete, so its flag must stay down in every pool (a consumer would wait, not read stale
+    pages), while the other chunks publish normally."""
+    P = Published(CASE, n_peers=2)
+    off, ps = CASE.chunk_offsets, CASE.page_size
+    bad_chunk = CASE.num_chunks - 2
+    P.pt[LAYER, (off[bad_chunk] + 3) // ps] = CASE.num_pages + 5
+    P.publish(range(CASE.num_chunks))
+    assert check_status() == WF_ERR_PAGE_OOB
+    assert check_status() == WF_OK
+    for f in P.flags:
+        row = f[LAYER, :CASE.num_chunks].cpu().tolist()
+        # a chunk that shares the bad page is incomplete too
+        bad = {c for c in range(CASE.num_chunks)
+               if off[c] // ps <= (off[bad_chunk] + 3) // ps <= (off[c + 1] - 1) // ps
+               and off[c + 1] > off[c]}
+        assert bad_chunk in bad
+        assert row == [0 if c in bad else GEN for c in range(CASE.num_chunks)]

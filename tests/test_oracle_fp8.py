@@ -88,6 +88,25 @@ def test_quantized_rows_hit_448_at_the_row_maximum_and_zero_rows_stay_zero():
     assert np.all(err <= bound)
 
 
+def test_rows_too_small_to_scale_are_stored_as_zeros():
+    """448 / amax overflows fp32 once amax < 448 / FLT_MAX (about 1.3e-36).  Such a row would
+    otherwise turn its zeros into 0 * inf = NaN codes; it is stored as signed zeros with scale
+    0, like a row of zeros.  Just above the threshold the row still quantizes normally."""
+    flt_max = float(np.finfo(np.float32).max)
+    threshold = 448.0 / flt_max
+    tiny = np.float32([1e-38, -5e-37, 0.0, 2.5e-38])                 # amax 5e-37 < threshold
+    big = np.float32([2.0e-36, 0.0, -1.0e-36, 3.0e-37])             # amax 2e-36 > threshold
+    assert np.abs(tiny).max() < threshold < np.abs(big).max()
+    codes, scale = fp8.quantize_rows(np.stack([tiny, big]))
+    assert scale[0] == 0 and [c & 0x7F for c in codes[0]] == [0, 0, 0, 0]
+    assert [c >> 7 for c in codes[0]] == [0, 1, 0, 0]                # signs kept
+    assert np.isfinite(scale[1]) and scale[1] > 0                    # a subnormal fp32 scale
+    assert (codes[1][0] & 0x7F) == 0x7E                              # the maximum hits 448
+    back = fp8.dequantize_rows_f32(codes, scale)
+    assert np.all(np.isfinite(back)) and not back[0].any()
+    assert abs(back[1][0] - big[0]) <= 2.0 ** -4 * abs(big[0])
+
+
 def test_dequantized_rows_are_the_bf16_rounding_of_the_fp32_product():
     codes = np.arange(256, dtype=np.uint8).reshape(2, 128)
     codes[(codes & 0x7F) == 0x7F] = 0              # no NaN codes

@@ -27,6 +27,7 @@ MUTANTS = [
     ("mantissa_of_four_bits", "(1.0 + m / 8.0)", "(1.0 + m / 16.0)"),
     ("decode_sign_dropped", "return np.where(c & 0x80, -out, out).astype(np.float32)",
      "return out.astype(np.float32)"),
+    ("overflowing_inverse_kept", "live = nz & np.isfinite(inv)", "live = nz"),
 ]
 
 PINS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

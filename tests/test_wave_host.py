@@ -128,3 +128,63 @@ def test_publish_argument_checks_without_a_gpu(abi):
     assert published(None) == abi.WF_ERR_INVALID_ARG
     assert published(FAKE + 1) == abi.WF_ERR_INVALID_ARG
     assert published(FAKE, splits=-2) == abi.WF_ERR_INVALID_ARG
+
+
+def _shared_alloc_worker(rank, world, port, results):
+    """Both pools and an FP8 pool exported from one fake allocation per rank: every tensor has
+    the same handle and its own offset, so the peer must map the allocation once, derive every
+    pointer from that one mapping, and close it once."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from block_causal_streaming_b200 import _abi
+        base = 0x7000_0000 + 0x100_0000 * rank
+        imports, closed = [], []
+
+        def export(ptr):
+            return (rank.to_bytes(4, "little") + base.to_bytes(8, "little")).ljust(64, b"\0"), \
+                int(ptr) - base
+
+        def imp(exported):
+            handle, off = exported
+            imports.append((handle[:4], off))
+            return 0x9000_0000 + 0x100_0000 * int.from_bytes(handle[:4], "little") + off
+
+        _abi.ipc_export, _abi.ipc_import, _abi.ipc_close = export, imp, closed.append
+        t = [torch.zeros(4, dtype=torch.int32) for _ in range(7)]
+        ptrs = {}
+
+        class T:                      # a tensor stand-in at a chosen address inside the block
+            def __init__(self, addr):
+                self.addr = addr
+
+            def data_ptr(self):
+                return self.addr
+        own = [T(base + 256 * i) for i in range(7)]
+        pools = wave.PublishedPools(own[0], own[1], own[2], fp8=own[3:])
+        other = 1 - rank
+        results[rank] = (pools.peer(other), pools.peer_fp8(other),
+                         pools.destinations_fp8([0, 1]), list(imports))
+        pools.close()
+        results[rank] = results[rank] + (list(closed),)
+        del t, ptrs
+    finally:
+        dist.destroy_process_group()
+
+
+def test_tensors_of_one_allocation_are_mapped_once():
+    world, port = 2, _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        results = m.dict()
+        mp.start_processes(_shared_alloc_worker, args=(world, port, results), nprocs=world,
+                           start_method="spawn", join=True)
+        res = dict(results)
+    for rank, (peer, peer_fp8, dests, imports, closed) in res.items():
+        other = 1 - rank
+        mapped = 0x9000_0000 + 0x100_0000 * other
+        assert len(imports) == 1 and len(closed) == 1                  # one allocation, once
+        assert peer == (mapped, mapped + 256, mapped + 512)
+        assert peer_fp8 == (mapped + 768, mapped + 1024, mapped + 1280, mapped + 1536,
+                            mapped + 512)                              # flags come last
+        assert dests == [peer_fp8]

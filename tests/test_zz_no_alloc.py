@@ -34,10 +34,16 @@ def test_noalloc_validation_without_a_gpu():
                                                   None) != WF_OK
 
 
-def _compare_two_calls(wl, splits):
-    from gpu_util import place
+def _compare_two_calls(wl, splits, rows=None, heads=None):
+    """Two calls of the no-alloc entry point must equal the workspace entry point bit for bit,
+    and the result must meet the parity bar against the oracle on its own (every element, or
+    the given (row, head) pairs)."""
+    import oracle
+    from gpu_util import assert_parity, place
     inp = make_inputs(wl)
     layer, q, _, _ = place(wl, inp, fill=float("nan"))
+    # the plan really splits, so the static scratch is in use
+    assert attn_workspace_size(layer.desc, wl.heads, wl.head_dim, splits) > 0
     ref = torch.empty_like(q)
     ref_lse = torch.empty(q.shape[1], q.shape[0], dtype=torch.float32, device=q.device)
     layer.forward(q, ref, lse=ref_lse, splits=splits)          # caller-workspace entry point
@@ -49,6 +55,14 @@ def _compare_two_calls(wl, splits):
         assert check_status() == WF_OK
         assert torch.equal(out, ref)
         assert torch.equal(lse, ref_lse)
+    scale = 1.0 / wl.head_dim ** 0.5
+    if rows is None:
+        want = oracle.attention(inp.q, inp.k, inp.v, wl.chunk_offsets, wl.num_ctx_chunks, scale)
+        assert_parity(out.float().cpu().numpy(), want, f"{wl.name} no-alloc")
+    else:
+        want = oracle.attention_rows(inp.q, inp.k, inp.v, wl.chunk_offsets, wl.num_ctx_chunks,
+                                     scale, rows, heads)
+        assert_parity(out[rows, heads].float().cpu().numpy(), want, f"{wl.name} no-alloc")
 
 
 @pytest.mark.gpu
@@ -62,7 +76,9 @@ def test_noalloc_matches_workspace_entry_on_two_calls(splits):
 def test_noalloc_matches_on_the_wave_parallel_rank_call():
     wl = WP_RANK0
     assert 0 < attn_workspace_size(_desc(wl), wl.heads, wl.head_dim, 0) <= SCRATCH_BYTES
-    _compare_two_calls(wl, 0)
+    from gpu_util import sample_rows
+    rows, heads = sample_rows(wl, per_chunk=16, seed=41)
+    _compare_two_calls(wl, 0, rows, heads)
 
 
 @pytest.mark.gpu
