@@ -78,6 +78,24 @@ def rows_flops(wl: Workload, rows, heads_per_row: int) -> int:
     return 4 * wl.head_dim * heads_per_row * total
 
 
+def workload_config(wl: Workload, world: int, split: bool) -> dict:
+    """The `config` object of a bench line: the workload, with its sizes, and how a step runs.
+    Both arms print the same object for the same workload."""
+    off, nctx = wl.chunk_offsets, wl.num_ctx_chunks
+    H, D = wl.heads, wl.head_dim
+    active = wl.num_chunks - nctx
+    # q, out, the appended K/V (read + written) and the K/V pages attention reads
+    touched_mb = (2 * wl.t_q * H * D + 4 * (off[-1] - off[nctx]) * H * D + 2 * off[-1] * H * D) \
+        * 2 / 1e6
+    return {"workload": wl.name, "heads": H, "head_dim": D, "t_q": wl.t_q, "t_kv": wl.t_kv,
+            "chunks": f"{nctx} ctx + {active} active x {off[nctx + 1] - off[nctx]}",
+            "page_size": wl.page_size,
+            "step": f"append {active} active chunks + attention"
+                    + (" (key splits + merge)" if split else ""),
+            "l2": f"inputs larger than L2 (~{touched_mb:.0f} MB touched per step vs 126 MB L2)",
+            "parallelism": f"replicas x{world}"}
+
+
 def kernel_hash() -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
@@ -277,11 +295,11 @@ def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     torch.cuda.synchronize(dev)
     for e in evs:
-        torch.sum(flush, out=sink)
+        torch.sum(flush, dim=(0,), out=sink)
         e[0].record(stream)
         quant()
         e[1].record(stream)
-        torch.sum(flush, out=sink)
+        torch.sum(flush, dim=(0,), out=sink)
         e[2].record(stream)
         dequant()
         e[3].record(stream)
@@ -433,8 +451,6 @@ def gpu_arm(args, world, rank, local):
         raise RuntimeError(f"device status after end-to-end run: {wf.strerror(rc)}")
 
     peaks, peak_src = load_peaks()
-    touched_mb = (2 * q.numel() + 4 * (off[-1] - off[nctx]) * H * D + 2 * off[-1] * H * D) \
-        * 2 / 1e6   # q, out, appended K/V (read + written), K/V pages read
     step_s = elapsed_max / args.steps
     value = aggregate(flop, world, step_s) / 1e12
     attn_avg_s = statistics.mean(attn_ms) / 1e3
@@ -445,14 +461,7 @@ def gpu_arm(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(step_s * 1e3, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)*0.5 bf16)",
-        "config": {"workload": wl.name, "heads": H, "head_dim": D, "t_q": wl.t_q,
-                   "t_kv": wl.t_kv, "chunks": f"{nctx} ctx + {len(active)} active x 4680",
-                   "page_size": wl.page_size,
-                   "step": f"append {len(active)} active chunks + attention"
-                           + (" (key splits + merge)" if split_used else ""),
-                   "l2": f"inputs larger than L2 (~{touched_mb:.0f} MB touched per step vs "
-                         "126 MB L2)",
-                   "parallelism": f"replicas x{world}"},
+        "config": workload_config(wl, world, split_used),
         "tokens_per_s": round(world * wl.t_q / step_s, 1),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "tensor",
@@ -510,8 +519,7 @@ def reference_arm(args, world, rank):
         "ms_per_step": round(1e3 * secs / args.steps, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1)*0.5 bf16)", "impl": "reference",
-        "config": {"workload": wl.name, "heads": wl.heads, "head_dim": wl.head_dim,
-                   "t_q": wl.t_q, "t_kv": wl.t_kv, "parallelism": "host cores"},
+        "config": workload_config(wl, world, wl is WP_RANK0),
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": os.cpu_count(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,

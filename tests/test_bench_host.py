@@ -92,3 +92,17 @@ def test_workload_selection():
     # one rank's call: one 4680-token chunk against 8 chunks of keys
     assert (WP_RANK0.t_q, WP_RANK0.t_kv, WP_RANK0.num_ctx_chunks) == (4680, 37440, 7)
     assert bench.attention_flops(WP_RANK0) == 4 * 128 * 12 * 4680 * 37440
+
+
+def test_both_arms_print_the_same_config(monkeypatch):
+    """The reference arm times the oracle on the workload the GPU arm runs, and says so with the
+    same `config` object (the GPU arm calls workload_config with the same arguments)."""
+    class A:
+        workload, steps, warmup, cpu_seconds = "wan13b_5step", 1, 3, 0.05
+    monkeypatch.setattr(bench, "oracle_sample",
+                        lambda wl, inp, target_s, seed=0: (1.0, {"rows": 4, "heads": wl.heads,
+                                                                 "seconds": 0.01, "flop": 1}))
+    line = bench.reference_arm(A, world=1, rank=0)
+    assert line["config"] == bench.workload_config(WAN13B_5STEP, 1, False)
+    assert line["config"]["chunks"] == "2 ctx + 5 active x 4680"
+    assert "633 MB" in line["config"]["l2"]
