@@ -289,10 +289,14 @@ def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
             wf.kv_dequant(*fp.tensors, layer.pool.k, layer.pool.v, 0, c, layer.page_tables,
                           layer.desc, stream)
 
+    def append_bf16():
+        layer.append_range(k, v, chunks, stream)
+
     for _ in range(warmup):
         quant()
         dequant()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        append_bf16()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
     torch.cuda.synchronize(dev)
     for e in evs:
         torch.sum(flush, dim=(0,), out=sink)
@@ -303,6 +307,10 @@ def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
         e[2].record(stream)
         dequant()
         e[3].record(stream)
+        torch.sum(flush, dim=(0,), out=sink)
+        e[4].record(stream)
+        append_bf16()
+        e[5].record(stream)
     torch.cuda.synchronize(dev)
     rc = wf.check_status()
     if rc != wf.WF_OK:
@@ -313,9 +321,13 @@ def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
     out = {"chunks": wl.num_chunks, "tokens": rows, "steps": steps,
            "bytes_bf16": bf16_bytes, "bytes_fp8": fp8_bytes,
            "bytes_ratio": round(fp8_bytes / bf16_bytes, 4), "peak_gbs": hbm_peak}
-    for name, (a, b) in (("append_fp8", (0, 1)), ("dequant", (2, 3))):
+    # the plain bf16 append of the same chunks, timed the same way: what one launch per chunk
+    # of this size reaches for a pure copy
+    for name, (a, b), nbytes in (("append_fp8", (0, 1), bf16_bytes + fp8_bytes),
+                                 ("dequant", (2, 3), bf16_bytes + fp8_bytes),
+                                 ("append_bf16_reference", (4, 5), 2 * bf16_bytes)):
         ms = statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
-        gbs = (bf16_bytes + fp8_bytes) / (ms / 1e3) / 1e9
+        gbs = nbytes / (ms / 1e3) / 1e9
         out[name] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4),
                      "launches": wl.num_chunks}
     return out

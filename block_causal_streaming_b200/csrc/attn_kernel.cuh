@@ -295,31 +295,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // convex combination of the visible values (V = 1 gives exactly 1).
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[BN / 2];
-        if (!masked) {
+        // P for column pairs [32 h, 32 h + 32): keys [64 h, 64 h + 64), bf16x2 into TMEM
+        // columns [32 h, 32 h + 32) of S_q.  (Publishing the first half early, so that P.V
+        // starts on it, measured 1-9 % slower.)
+        auto p_half = [&](int h) {
+          if (!masked) {
   #pragma unroll
-          for (int i = 0; i < BN / 2; ++i) {
-            const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2x2, negm);
-            float2 e;
-            if ((i & 7) < WF_EXP2_POLY_EIGHTHS) {
-              e = exp2_poly2(x);
-            } else {
-              e.x = ex2_approx(x.x);
-              e.y = ex2_approx(x.y);
+            for (int i = 32 * h; i < 32 * h + 32; ++i) {
+              const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2x2, negm);
+              float2 e;
+              if ((i & 7) < WF_EXP2_POLY_EIGHTHS) {
+                e = exp2_poly2(x);
+              } else {
+                e.x = ex2_approx(x.x);
+                e.y = ex2_approx(x.y);
+              }
+              pk[i] = pack_bf16x2(e.x, e.y);
+              acc[i & 3] = add_bf16x2(acc[i & 3], pk[i]);
             }
-            pk[i] = pack_bf16x2(e.x, e.y);
-            acc[i & 3] = add_bf16x2(acc[i & 3], pk[i]);
-          }
-        } else {
+          } else {
   #pragma unroll
-          for (int i = 0; i < BN / 2; ++i) {
-            const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2x2, negm);
-            pk[i] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
-            acc[i & 3] = add_bf16x2(acc[i & 3], pk[i]);
+            for (int i = 32 * h; i < 32 * h + 32; ++i) {
+              const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2x2, negm);
+              pk[i] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
+              acc[i & 3] = add_bf16x2(acc[i & 3], pk[i]);
+            }
           }
-        }
-  #pragma unroll
-        for (int h = 0; h < BN / 64; ++h)
           tmem_st32(tS + 32u * h, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h]));
+        };
+        p_half(0);
+        p_half(1);
         l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
         tmem_wait_st();
         tc_fence_before();
@@ -507,11 +512,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint64_t dv = dv0 + ((static_cast<uint32_t>(slotv) * KTILE) >> 4);
   #pragma unroll 1
         for (int q = 0; q < kNQT && ok; ++q) {
+          const uint32_t pa = tmem + static_cast<uint32_t>(q * 128);
+          const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
           ok = mbar_wait(bar(L::B_P + q), j & 1, w);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t pa = tmem + static_cast<uint32_t>(q * 128);
-          const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
   #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
             umma_ts(od, pa + 8u * kk, dv + ((kk * 2048u) >> 4), idesc_pv,

@@ -704,14 +704,24 @@ int fp8_chunk_args(const wf_kv_pool_fp8_t* pool, int layer, int chunk, const int
   *t0 = wf->chunk_offsets[chunk];
   *rows = wf->chunk_offsets[chunk + 1] - *t0;
   *row = page_table + static_cast<int64_t>(layer) * wf->max_pages_per_seq;
+  // the quantizer indexes its threads over the (token, head) rows of both tensors with 32-bit
+  // integers
+  if (8 * static_cast<int64_t>(*rows) * pool->num_heads >= (int64_t{1} << 30)) return WF_ERR_SHAPE;
   return WF_OK;
 }
 
-// One warp per token.
-int fp8_blocks(const DeviceState* d, int rows) {
-  const int64_t warps = rows;
+// Quantization: kQuantLanes threads per (token, head) row of each tensor.
+int quant_blocks(const DeviceState* d, int rows, int heads) {
+  const int64_t threads = 2 * wfk::kQuantLanes * static_cast<int64_t>(rows) * heads;
+  const int64_t blocks = (threads + wfk::kFp8Threads - 1) / wfk::kFp8Threads;
+  const int64_t cap = static_cast<int64_t>(d->num_sms) * 16;
+  return static_cast<int>(blocks < cap ? blocks : cap);
+}
+
+// Dequantization: one warp per token.
+int dequant_blocks(const DeviceState* d, int rows) {
   const int per_block = wfk::kFp8Threads / 32;
-  int64_t blocks = (warps + per_block - 1) / per_block;
+  const int64_t blocks = (static_cast<int64_t>(rows) + per_block - 1) / per_block;
   const int64_t cap = static_cast<int64_t>(d->num_sms) * 8;   // 64 warps per SM in flight
   return static_cast<int>(blocks < cap ? blocks : cap);
 }
@@ -746,7 +756,7 @@ int launch_quant(const wf_kv_pool_fp8_t* pool, const wf_fp8_dst_t* peers, int nu
   for (int i = 0; i < num_peers; ++i)
     p.dst[1 + i] = {static_cast<uint8_t*>(peers[i].k_codes),
                     static_cast<uint8_t*>(peers[i].v_codes), peers[i].k_scale, peers[i].v_scale};
-  const int blocks = fp8_blocks(d, rows);
+  const int blocks = quant_blocks(d, rows, pool->num_heads);
   if (pool->head_dim == 128)
     wfk::wf_quant_append_kernel<128><<<blocks, wfk::kFp8Threads, 0, s>>>(p);
   else
@@ -781,7 +791,7 @@ int launch_dequant(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int t0,
   p.grid_abort = d->abort_word;
   p.launch_id = g_launch_counter.fetch_add(1);
   if (p.launch_id == 0) p.launch_id = g_launch_counter.fetch_add(1);
-  const int blocks = fp8_blocks(d, rows);
+  const int blocks = dequant_blocks(d, rows);
   const bool wait = flag != nullptr;
   if (src->head_dim == 128 && !wait)
     wfk::wf_dequant_kernel<128, false><<<blocks, wfk::kFp8Threads, 0, s>>>(p);
