@@ -12,7 +12,9 @@ The product is the C-ABI library ``libwf_b200.so`` (declared in ``include/wf.h``
 * ``wf_kv_append_fp8`` / ``wf_kv_dequant`` -- a chunk's K/V as e4m3 codes with per-(token, head)
   scales (half the bytes to move), and their conversion back into the bf16 pool;
   ``wf_kv_append_publish_fp8`` / ``wf_kv_dequant_published`` publish those codes into other GPUs'
-  FP8 pools with a generation flag, and convert a published chunk once its flag is up.
+  FP8 pools with a generation flag, and convert a published chunk once its flag is up;
+* ``wf_qk_quantize_i8`` / ``wf_attn_forward_i8`` -- the INT8 tier: smoothed int8 K and int8 Q
+  with per-128-row scales, QK^T as an integer product on the tensor core.
 
 This package is its thin Python binding (ctypes, argument marshalling only), a small helper that
 owns the paged pools of one layer (:mod:`.layer`), the round-by-round planner of a streaming
@@ -27,7 +29,8 @@ _ABI_NAMES = (
     "selftest_timeout", "attn_forward_split", "attn_workspace_size",
     "attn_forward_split_noalloc", "kv_append_publish", "attn_forward_published", "ipc_export",
     "ipc_import", "ipc_close", "PoolDst", "kv_append_fp8", "kv_dequant", "KvPoolFp8",
-    "kv_append_publish_fp8", "kv_dequant_published", "Fp8Dst",
+    "kv_append_publish_fp8", "kv_dequant_published", "Fp8Dst", "qk_i8_sizes", "qk_quantize_i8",
+    "attn_forward_i8", "QkI8",
 )
 __all__ = list(_ABI_NAMES)
 

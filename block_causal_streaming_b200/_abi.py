@@ -30,6 +30,7 @@ EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror",
             "wf_attn_forward_split_noalloc", "wf_kv_append_publish", "wf_attn_forward_published",
             "wf_ipc_export", "wf_ipc_import", "wf_ipc_close", "wf_kv_append_fp8",
             "wf_kv_dequant", "wf_kv_append_publish_fp8", "wf_kv_dequant_published",
+            "wf_qk_i8_sizes", "wf_qk_quantize_i8", "wf_attn_forward_i8",
             "wf_window_slots", "wf_window_round")
 
 
@@ -50,6 +51,13 @@ class Fp8Dst(ctypes.Structure):
     _fields_ = [("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
                 ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
                 ("flags", ctypes.c_void_p)]
+
+
+class QkI8(ctypes.Structure):
+    """wf_qk_i8_t: the quantized Q and K' of the INT8 tier (device pointers)."""
+    _fields_ = [("q_codes", ctypes.c_void_p), ("q_scale", ctypes.c_void_p),
+                ("k_codes", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
+                ("k_mean", ctypes.c_void_p), ("k_sum", ctypes.c_void_p)]
 
 
 class KvPool(ctypes.Structure):
@@ -153,6 +161,16 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
                                             i32, i32, ctypes.POINTER(ctypes.c_int32),
                                             ctypes.POINTER(Wavefront), vp, ctypes.c_uint32, vp]
     lib.wf_kv_dequant_published.restype = i32
+    lib.wf_qk_i8_sizes.argtypes = [ctypes.POINTER(Wavefront), i32, i32,
+                                   ctypes.POINTER(ctypes.c_size_t)]
+    lib.wf_qk_i8_sizes.restype = i32
+    lib.wf_qk_quantize_i8.argtypes = [vp, ctypes.POINTER(KvPool), ctypes.POINTER(ctypes.c_int32),
+                                      ctypes.POINTER(Wavefront), ctypes.POINTER(QkI8), vp]
+    lib.wf_qk_quantize_i8.restype = i32
+    lib.wf_attn_forward_i8.argtypes = [ctypes.POINTER(QkI8), ctypes.POINTER(KvPool),
+                                       ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(Wavefront),
+                                       f32, vp, ctypes.POINTER(ctypes.c_float), vp]
+    lib.wf_attn_forward_i8.restype = i32
     lib.wf_window_slots.argtypes = [ctypes.POINTER(WindowC), ctypes.POINTER(ctypes.c_int32),
                                     ctypes.POINTER(ctypes.c_int64)]
     lib.wf_window_slots.restype = i32
@@ -247,7 +265,7 @@ def _check_queries(q, out, lse, wf: "WavefrontDesc", H: int, D: int):
 def _check_tensor(t, name: str, dtype_name: str):
     import torch
     want = {"bf16": (torch.bfloat16,), "i32": (torch.int32,), "f32": (torch.float32,),
-            "u8": (torch.uint8,),
+            "u8": (torch.uint8,), "i8": (torch.int8,), "f64": (torch.float64,),
             "u32": (torch.int32, torch.uint32)}[dtype_name]      # flag words: any 32-bit int
     if t.dtype not in want:
         raise TypeError(f"{name}: expected {want[0]}, got {t.dtype}")
@@ -415,6 +433,76 @@ def kv_dequant_published(k_codes, v_codes, k_scale, v_scale, k_pool, v_pool, lay
                                      int(generation) & 0xFFFFFFFF, _stream_handle(stream))
     if rc != WF_OK:
         raise WfError(rc, "wf_kv_dequant_published")
+
+
+QK_I8_FIELDS = ("q_codes", "q_scale", "k_codes", "k_scale", "k_mean", "k_sum")
+
+
+def qk_i8_sizes(wf: WavefrontDesc, num_heads: int, head_dim: int):
+    """wf_qk_i8_sizes: byte sizes of the six buffers of the INT8 tier, in QK_I8_FIELDS order."""
+    sizes = (ctypes.c_size_t * 6)()
+    rc = lib.wf_qk_i8_sizes(ctypes.byref(wf.c), int(num_heads), int(head_dim), sizes)
+    if rc != WF_OK:
+        raise WfError(rc, "wf_qk_i8_sizes")
+    return [int(x) for x in sizes]
+
+
+def _qk_struct(qk) -> QkI8:
+    """qk: a mapping / object with the six QK_I8_FIELDS device tensors."""
+    get = (lambda n: qk[n]) if isinstance(qk, dict) else (lambda n: getattr(qk, n))
+    for n, d in zip(QK_I8_FIELDS, ("i8", "f32", "i8", "f32", "f32", "f64")):
+        _check_tensor(get(n), n, d)
+    return QkI8(*[get(n).data_ptr() for n in QK_I8_FIELDS])
+
+
+def qk_quantize_i8(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, qk,
+                   stream=None) -> None:
+    """wf_qk_quantize_i8: int8 Q (from q) and K' (from the K pool) with their scales into qk."""
+    _, _, H, D = _pool_shape(k_pool, v_pool)
+    _check_queries(q, q, None, wf, H, D)
+    _check_page_table_row(page_table_row, wf)
+    sizes = qk_i8_sizes(wf, H, D)
+    get = (lambda n: qk[n]) if isinstance(qk, dict) else (lambda n: getattr(qk, n))
+    for n, sz in zip(QK_I8_FIELDS, sizes):
+        t = get(n)
+        if t.numel() * t.element_size() < sz:
+            raise ValueError(f"{n}: {t.numel() * t.element_size()} bytes, needs {sz}")
+    for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"),
+                    (page_table_row, "page_table_row", "i32")):
+        _check_tensor(t, n, d)
+    pool = _pool_struct(k_pool, v_pool)
+    s = _qk_struct(qk)
+    rc = lib.wf_qk_quantize_i8(q.data_ptr(), ctypes.byref(pool),
+                               ctypes.cast(ctypes.c_void_p(page_table_row.data_ptr()),
+                                           ctypes.POINTER(ctypes.c_int32)),
+                               ctypes.byref(wf.c), ctypes.byref(s), _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_qk_quantize_i8")
+
+
+def attn_forward_i8(qk, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: float, out,
+                    lse=None, stream=None) -> None:
+    """wf_attn_forward_i8: block-causal attention on the quantized Q / K' of qk, V from v_pool."""
+    _, _, H, D = _pool_shape(k_pool, v_pool)
+    _check_queries(out, out, lse, wf, H, D)
+    _check_page_table_row(page_table_row, wf)
+    for t, n, d in ((out, "out", "bf16"), (v_pool, "v_pool", "bf16"),
+                    (page_table_row, "page_table_row", "i32")):
+        _check_tensor(t, n, d)
+    if lse is not None:
+        _check_tensor(lse, "lse", "f32")
+    pool = _pool_struct(k_pool, v_pool)
+    s = _qk_struct(qk)
+    rc = lib.wf_attn_forward_i8(ctypes.byref(s), ctypes.byref(pool),
+                                ctypes.cast(ctypes.c_void_p(page_table_row.data_ptr()),
+                                            ctypes.POINTER(ctypes.c_int32)),
+                                ctypes.byref(wf.c), float(scale), out.data_ptr(),
+                                ctypes.cast(ctypes.c_void_p(lse.data_ptr()),
+                                            ctypes.POINTER(ctypes.c_float))
+                                if lse is not None else None,
+                                _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_attn_forward_i8")
 
 
 def attn_forward(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: float, out,

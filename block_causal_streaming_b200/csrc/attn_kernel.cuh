@@ -51,6 +51,8 @@
 
 #include <cuda_bf16.h>
 
+#include <cfloat>
+
 #include "sm100.cuh"
 
 namespace wfk {
@@ -107,6 +109,11 @@ struct AttnParams {
   unsigned flag_gen;
   int nchunks;
   int chunk_end[kMaxQChunks];
+  // INT8 tier (kI8): tm_q / tm_k describe int8 Q and K' codes ([rows][H][D], K' contiguous in
+  // logical key order), with one scale per (128 rows, head): q_scale [H][nqt], k_scale [H][nkb].
+  const float* q_scale;
+  const float* k_scale;
+  int nqt, nkb;
 };
 
 __device__ __forceinline__ int kv_end_of_row(const AttnParams& p, int r) {
@@ -136,13 +143,16 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-template <int D>
+// kI8: Q and K tiles hold int8 codes (one 128-byte row per query / key at head_dim 128), V
+// stays bf16; the 32 KB Q saves go to a sixth ring slot.
+template <int D, bool kI8 = false>
 struct AttnSmem {
   static constexpr int BN = kBN;
-  static constexpr int DH = D / 64;                      // 128-byte halves of a row
-  static constexpr int NS = WF_KV_RING_KB * 1024 / (int)(DH * BN * 128);   // K/V ring slots
+  static constexpr int DH = D / 64;                      // 128-byte halves of a bf16 row
+  static constexpr int NS = (WF_KV_RING_KB + (kI8 ? 32 : 0)) * 1024 / (int)(DH * BN * 128);
   static constexpr uint32_t QHALF = kBM * 128u;          // 128 rows x 128 B, 128B-swizzled
-  static constexpr uint32_t QTILE = DH * QHALF;
+  static constexpr uint32_t QTILE = kI8 ? QHALF : DH * QHALF;
+  static constexpr uint32_t KBYTES = kI8 ? BN * 128u : DH * BN * 128u;   // bytes a K tile loads
   static constexpr uint32_t KHALF = BN * 128u;           // BN rows x 128 B
   static constexpr uint32_t KTILE = DH * KHALF;          // one K or V tile
   static constexpr uint32_t Q_OFF = 0;
@@ -160,10 +170,13 @@ struct AttnSmem {
 
 // kWaitPublished: wait for the publication flags of the chunks (AttnParams::flags) before
 // loading their keys; a separate instantiation so the plain kernel carries none of that code.
-template <int D, bool kWaitPublished = false>
+// kI8: the INT8 tier -- S = Q_i8 K_i8^T on the tensor core (kind::i8, s32 in TMEM), each S tile
+// scaled by scale_q x scale_k in the softmax; P and P.V as in the bf16 kernel.
+template <int D, bool kWaitPublished = false, bool kI8 = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     wf_attn_fwd_kernel(const __grid_constant__ AttnParams p) {
-  using L = AttnSmem<D>;
+  static_assert(!kI8 || (D == 128 && !kWaitPublished), "the INT8 tier runs head_dim 128");
+  using L = AttnSmem<D, kI8>;
   constexpr int BN = L::BN, DH = L::DH, NS = L::NS;
   constexpr uint32_t QTILE = L::QTILE, QHALF = L::QHALF, KTILE = L::KTILE, KHALF = L::KHALF;
 
@@ -225,12 +238,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
       const uint32_t tS = tmem + lane_off + static_cast<uint32_t>(q * 128);
       const uint32_t tO = tmem + lane_off + 256u + static_cast<uint32_t>(q * D);
-      const float sl2 = p.sl2;
+      const float sl2 = kI8 ? p.sl2 * __ldg(p.q_scale + head * p.nqt + (m0 + q * kBM) / kBM)
+                            : p.sl2;
       float m2 = -INFINITY;   // running max of the base-2 logits in use
       float l = 0.f;          // running sum of exp2(t - m2)
       bool ok = true;
-      const float2 sl2x2 = make_float2(sl2, sl2);
+      float2 sl2x2 = make_float2(sl2, sl2);
       for (int j = 0; j < nk; ++j) {
+        // INT8 tier: the tile's K scale is loaded before the wait for S, which hides its latency
+        const float dk = kI8 ? __ldg(p.k_scale + head * p.nkb + kb + j) : 0.f;
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_S + q), j & 1, w));
         if (!ok) break;
         tc_fence_after();
@@ -241,8 +257,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int c = 0; c < BN / 32; ++c)
             tmem_ld32(tS + 32u * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
           tmem_wait_ld();
+          if (kI8) {
+            // s32 -> fp32, exact: |S| <= 128 x 127^2 < 2^24.  (Reading the bits of
+            // 1.5 x 2^23 + S as a float and subtracting 1.5 x 2^23 measured 3 % slower.)
   #pragma unroll
-          for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
+            for (int c = 0; c < BN; ++c) s[c] = static_cast<float>(static_cast<int>(r[c]));
+          } else {
+  #pragma unroll
+            for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
+          }
+        }
+        float tsl2 = sl2;     // logit scale of this tile
+        if (kI8) {
+          // scale_q x scale_k x scale x log2 e; a zero scale (a block of zeros) is kept
+          // positive so masked columns stay -inf rather than 0 x inf
+          tsl2 = fmaxf(sl2 * dk, FLT_MIN);
+          sl2x2 = make_float2(tsl2, tsl2);
         }
         const int lim = n_r - (kb + j) * BN;                // visible columns of this tile
         const bool masked = lim < BN;
@@ -258,7 +288,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (c + 4 < BN) mx2 = max3(mx2, s[c + 4], s[c + 5]);
           if (c + 6 < BN) mx3 = max3(mx3, s[c + 6], s[c + 7]);
         }
-        const float tmax = max3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
+        const float tmax = max3(mx0, mx1, fmaxf(mx2, mx3)) * tsl2;
         // Move the reference max only when the new one exceeds it by more than 2^8: O and l both
         // stay expressed against the same stale reference, so O / l is unchanged, and every
         // exp2(t - m2) stays <= 256.
@@ -391,7 +421,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   #pragma unroll
         for (int qt = 0; qt < kNQT; ++qt)
   #pragma unroll
-          for (int h = 0; h < DH; ++h)
+          for (int h = 0; h < (kI8 ? 1 : DH); ++h)     // int8: one 128-byte box per row
             tma_load_3d(base + L::Q_OFF + qt * QTILE + h * QHALF, &p.tm_q, 64 * h, head,
                         m0 + qt * kBM, bar(L::B_Q));
       }
@@ -423,9 +453,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int it = 2 * j + kv, slot = it % NS;
             ok = mbar_wait(bar(L::B_KVE + slot), ((it / NS) & 1) ^ 1, w);
             if (!ok) break;
-            mbar_arrive_expect_tx(bar(L::B_KVF + slot), KTILE);
             const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
             const uint32_t dst = base + L::KV_OFF + slot * KTILE;
+            if (kI8 && kv == 0) {
+              // int8 K' codes are contiguous in logical key order: one box of BN keys
+              mbar_arrive_expect_tx(bar(L::B_KVF + slot), L::KBYTES);
+              tma_load_3d(dst, map, 0, head, (kb + j) * BN, bar(L::B_KVF + slot));
+              last_it[slot] = it;
+              continue;
+            }
+            mbar_arrive_expect_tx(bar(L::B_KVF + slot), KTILE);
   #pragma unroll
             for (int b = 0; b < BN / 16; ++b) {
               if (b < nb) {
@@ -473,7 +510,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // instruction only a compile-time offset (16-byte units) is added to the start-address
       // field, so one MMA costs a few instructions to issue -- the tensor core retires a
       // 128 x BN x 16 step in BN/2 cycles and must not wait for the issuer.
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, BN, 0, 0);   // Q, K both K-major
+      constexpr uint32_t idesc_qk = kI8 ? idesc_s8_s32(kBM, BN)      // Q, K both K-major
+                                        : idesc_bf16_f32(kBM, BN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);     // P (TMEM), V MN-major
       const uint64_t dq0 = smem_desc_sw128(base + L::Q_OFF, 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(base + L::KV_OFF, 16, 1024);
@@ -487,10 +525,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint64_t dk = dk0 + ((static_cast<uint32_t>(slot) * KTILE) >> 4);
         const uint32_t sd = tmem + static_cast<uint32_t>(q * 128);
         const uint64_t dq = dq0 + ((static_cast<uint32_t>(q) * QTILE) >> 4);
+        if (kI8) {
+          // D int8 values = one 128-byte swizzle row; K-steps of 32 values (32 bytes)
   #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss(sd, dq + (((kk / 4) * QHALF + (kk % 4) * 32) >> 4),
-                  dk + (((kk / 4) * KHALF + (kk % 4) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 32; ++kk)
+            umma_ss_i8(sd, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), idesc_qk,
+                       kk > 0 ? 1u : 0u);
+        } else {
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_ss(sd, dq + (((kk / 4) * QHALF + (kk % 4) * 32) >> 4),
+                    dk + (((kk / 4) * KHALF + (kk % 4) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+        }
         umma_commit(bar(L::B_S + q));
       };
       auto wait_k = [&](int j) -> bool {

@@ -16,6 +16,7 @@
 #include "attn_kernel.cuh"
 #include "combine_kernel.cuh"
 #include "fp8_kernel.cuh"
+#include "i8_kernel.cuh"
 #include "publish_kernel.cuh"
 
 // First error any kernel of this library recorded on this device (0 = none); cleared by
@@ -81,7 +82,10 @@ int device_state(DeviceState** out) {
                                  wfk::AttnSmem<128>::ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<64, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 wfk::AttnSmem<64>::ALLOC) != cudaSuccess) {
+                                 wfk::AttnSmem<64>::ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<128, false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 wfk::AttnSmem<128, true>::ALLOC) != cudaSuccess) {
           cudaGetLastError();
           return WF_ERR_CUDA;
         }
@@ -180,6 +184,21 @@ bool encode_rows(CUtensorMap* map, const void* ptr, int D, int H, int64_t rows, 
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// uint8 tensor (D, H, rows) with row stride H*D bytes, 128B swizzle, box (128, 1, box_rows): the
+// int8 Q and K' codes of the INT8 tier (D = 128 bytes per row).
+bool encode_rows_u8(CUtensorMap* map, const void* ptr, int D, int H, int64_t rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H) * D};
+  const cuuint32_t box[3] = {128u, 1u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int gcd_int(int a, int b) {
@@ -898,6 +917,107 @@ int wf_kv_dequant_published(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst
   if (rows == 0) return WF_OK;
   return launch_dequant(src, dst, t0, rows, row, flags_row + chunk, generation,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+int wf_qk_i8_sizes(const wf_wavefront_t* wf, int num_heads, int head_dim, size_t sizes[6]) {
+  if (wf == nullptr || sizes == nullptr || num_heads < 1 || head_dim != 128 ||
+      wf->chunk_offsets == nullptr || wf->num_chunks < 1 || wf->num_chunks > WF_MAX_CHUNKS ||
+      wf->num_ctx_chunks < 0 || wf->num_ctx_chunks >= wf->num_chunks)
+    return head_dim != 128 && wf != nullptr && sizes != nullptr ? WF_ERR_SHAPE
+                                                                 : WF_ERR_INVALID_ARG;
+  const int64_t t_kv = wf->chunk_offsets[wf->num_chunks];
+  const int64_t t_q = t_kv - wf->chunk_offsets[wf->num_ctx_chunks];
+  const int64_t hd = static_cast<int64_t>(num_heads) * head_dim;
+  sizes[0] = static_cast<size_t>(t_q * hd);                                       // q_codes
+  sizes[1] = static_cast<size_t>(num_heads * ((t_q + 127) / 128)) * sizeof(float);  // q_scale
+  sizes[2] = static_cast<size_t>(t_kv * hd);                                      // k_codes
+  sizes[3] = static_cast<size_t>(num_heads * ((t_kv + 127) / 128)) * sizeof(float); // k_scale
+  sizes[4] = static_cast<size_t>(hd) * sizeof(float);                             // k_mean
+  sizes[5] = static_cast<size_t>(hd) * sizeof(double);                            // k_sum
+  return WF_OK;
+}
+
+int wf_qk_quantize_i8(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* page_table_row,
+                      const wf_wavefront_t* wf, const wf_qk_i8_t* qk, wf_stream_t stream) {
+  int rc = validate_pool(kv_pages);
+  if (rc) return rc;
+  if (kv_pages->head_dim != 128) return WF_ERR_SHAPE;
+  int t_kv = 0;
+  rc = validate_wavefront(wf, kv_pages, &t_kv);
+  if (rc) return rc;
+  if (wf->num_ctx_chunks >= wf->num_chunks) return WF_ERR_SHAPE;
+  const int t_q = t_kv - wf->chunk_offsets[wf->num_ctx_chunks];
+  if (t_q == 0) return WF_OK;
+  if (q == nullptr || qk == nullptr || page_table_row == nullptr || !aligned16(q) ||
+      qk->q_codes == nullptr || qk->k_codes == nullptr || qk->q_scale == nullptr ||
+      qk->k_scale == nullptr || qk->k_mean == nullptr || qk->k_sum == nullptr ||
+      !aligned16(qk->q_codes) || !aligned16(qk->k_codes) || !aligned16(qk->k_mean) ||
+      (reinterpret_cast<uintptr_t>(qk->k_sum) & 7u) ||
+      (reinterpret_cast<uintptr_t>(qk->q_scale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(qk->k_scale) & 3u))
+    return WF_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  rc = device_state(&d);
+  if (rc) return rc;
+  const int H = kv_pages->num_heads, D = 128, cols = H * D;
+  wfk::QkI8Params p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_pool = static_cast<const __nv_bfloat16*>(kv_pages->k_pool);
+  p.pt_row = page_table_row;
+  p.q_codes = static_cast<int8_t*>(qk->q_codes);
+  p.q_scale = qk->q_scale;
+  p.k_codes = static_cast<int8_t*>(qk->k_codes);
+  p.k_scale = qk->k_scale;
+  p.k_mean = qk->k_mean;
+  p.k_sum = qk->k_sum;
+  p.status = d->status;
+  p.T_q = t_q;
+  p.T_kv = t_kv;
+  p.H = H;
+  p.page_size = kv_pages->page_size;
+  p.num_pages = kv_pages->num_pages;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(qk->k_sum, 0, static_cast<size_t>(cols) * sizeof(double), s) != cudaSuccess)
+    return WF_ERR_CUDA;
+  int per = (t_kv + 4 * d->num_sms - 1) / (4 * d->num_sms);
+  per = std::max(1, std::min(per, wfk::kKmeanMaxPer));
+  wfk::wf_kmean_kernel<128><<<(t_kv + per - 1) / per, wfk::kKmeanThreads, 0, s>>>(p, per);
+  wfk::wf_kmean_finalize<<<(cols + 255) / 256, 256, 0, s>>>(p, cols);
+  wfk::wf_block_quant_kernel<128, true>
+      <<<dim3((t_kv + wfk::kI8Block - 1) / wfk::kI8Block, H), wfk::kQuantI8Threads, 0, s>>>(p);
+  wfk::wf_block_quant_kernel<128, false>
+      <<<dim3((t_q + wfk::kI8Block - 1) / wfk::kI8Block, H), wfk::kQuantI8Threads, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_attn_forward_i8(const wf_qk_i8_t* qk, const wf_kv_pool_t* kv_pages,
+                       const int32_t* page_table_row, const wf_wavefront_t* wf, float scale,
+                       void* out, float* lse_or_null, wf_stream_t stream) {
+  if (qk == nullptr || qk->q_codes == nullptr || qk->k_codes == nullptr ||
+      qk->q_scale == nullptr || qk->k_scale == nullptr || !aligned16(qk->k_codes))
+    return WF_ERR_INVALID_ARG;
+  if (kv_pages != nullptr && kv_pages->head_dim != 128) return WF_ERR_SHAPE;
+  AttnLaunch L;
+  int rc = prepare_attention(qk->q_codes, kv_pages, page_table_row, wf, scale, out, lse_or_null,
+                             &L);
+  if (rc || L.p.T_q == 0) return rc;
+  wfk::AttnParams& p = L.p;
+  const int t_kv = wf->chunk_offsets[wf->num_chunks];
+  if (!encode_rows_u8(&p.tm_q, qk->q_codes, 128, p.H, p.T_q, wfk::kBM) ||
+      !encode_rows_u8(&p.tm_k, qk->k_codes, 128, p.H, t_kv, wfk::kBN))
+    return WF_ERR_CUDA;
+  p.q_scale = qk->q_scale;
+  p.k_scale = qk->k_scale;
+  p.nqt = (p.T_q + wfk::kBM - 1) / wfk::kBM;
+  p.nkb = (t_kv + wfk::kBN - 1) / wfk::kBN;
+  p.launch_id = g_launch_counter.fetch_add(1);
+  if (p.launch_id == 0) p.launch_id = g_launch_counter.fetch_add(1);
+  const unsigned g = static_cast<unsigned>(static_cast<int64_t>(p.n_pairs) * p.H);
+  wfk::wf_attn_fwd_kernel<128, false, true>
+      <<<g, wfk::kAttnThreads, wfk::AttnSmem<128, true>::ALLOC,
+         reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
 int wf_selftest_timeout(unsigned timeout_us, wf_stream_t stream) {

@@ -47,6 +47,25 @@ class PagedPoolFp8:
         return self.k_codes, self.v_codes, self.k_scale, self.v_scale
 
 
+class QkI8Buffers:
+    """The device buffers of the INT8 attention tier for one wavefront shape (see
+    ``wf_qk_quantize_i8``): int8 Q and K' codes, their per-128-row scales, the key mean and its
+    fp64 scratch."""
+
+    def __init__(self, desc, heads: int, head_dim: int, device="cuda"):
+        from . import _abi
+        sizes = _abi.qk_i8_sizes(desc, heads, head_dim)
+        off = desc.chunk_offsets
+        t_kv, t_q = off[-1], off[-1] - off[desc.num_ctx_chunks]
+        self.q_codes = torch.empty(t_q, heads, head_dim, dtype=torch.int8, device=device)
+        self.q_scale = torch.empty(sizes[1] // 4, dtype=torch.float32, device=device)
+        self.k_codes = torch.empty(t_kv, heads, head_dim, dtype=torch.int8, device=device)
+        self.k_scale = torch.empty(sizes[3] // 4, dtype=torch.float32, device=device)
+        self.k_mean = torch.empty(heads, head_dim, dtype=torch.float32, device=device)
+        self.k_sum = torch.empty(heads, head_dim, dtype=torch.float64, device=device)
+        self.heads = heads
+
+
 class WavefrontLayer:
     """One layer of a wavefront: its descriptor and its page-table rows.
 
@@ -81,6 +100,18 @@ class WavefrontLayer:
         for c in chunks:
             a, b = self.chunk_offsets[c], self.chunk_offsets[c + 1]
             self.append(c, k_all[a:b], v_all[a:b], stream)
+
+    def forward_i8(self, q: torch.Tensor, out: torch.Tensor, qk: "QkI8Buffers",
+                   scale: Optional[float] = None, lse: Optional[torch.Tensor] = None,
+                   stream=None) -> None:
+        """The INT8 tier: quantize q and this layer's keys into ``qk``, then attend."""
+        from . import _abi
+        if scale is None:
+            scale = 1.0 / math.sqrt(self.pool.head_dim)
+        row = self.page_tables[self.layer]
+        _abi.qk_quantize_i8(q, self.pool.k, self.pool.v, row, self.desc, qk, stream)
+        _abi.attn_forward_i8(qk, self.pool.k, self.pool.v, row, self.desc, scale, out, lse,
+                             stream)
 
     def forward(self, q: torch.Tensor, out: torch.Tensor, scale: Optional[float] = None,
                 lse: Optional[torch.Tensor] = None, stream=None,

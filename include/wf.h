@@ -319,6 +319,50 @@ int wf_kv_dequant_published(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst
                             const uint32_t* flags_row, uint32_t generation, wf_stream_t stream);
 
 /*
+ * INT8 attention tier (Sage-like).  The pages name SageAttention with W8A8 as the fast attention
+ * backend (GitHub README, results table, "Sage . causal . paged" rows; KipQuest abstract) and give
+ * no internals; the tier built here, in two calls:
+ *   wf_qk_quantize_i8  mu = mean of the layer's keys per (head, channel) over all T_kv tokens
+ *                      (exact fp64 sum, fp64 division, one fp32 rounding); K' = fp32(K - mu),
+ *                      which shifts every logit of a query row by one constant and so leaves the
+ *                      softmax unchanged; then Q per (128 query rows, head) and K' per (128 keys,
+ *                      head), counted from row / key 0, as int8 codes with scale = amax / 127:
+ *                      code = clamp(round_half_even(x * (127 / amax)), -127, 127), fp32 steps
+ *                      (a block of zeros, or one whose 127 / amax overflows, gets scale 0).
+ *   wf_attn_forward_i8 the block-causal attention of wf_attn_forward with
+ *                      S = scale * scale_q * scale_k * (Q_i8 . K_i8) -- an exact integer product
+ *                      on the tensor core -- and P.V in bf16 over the unquantized V pages.
+ * Head dimension 128 only (WF_ERR_SHAPE otherwise).  All buffers are caller-owned device memory,
+ * sized by wf_qk_i8_sizes; codes are int8 [rows][H][D] with K' in logical key order (contiguous,
+ * no page table), scales fp32 [H][ceil(rows / 128)].
+ * --------------------------------------------------------------------------------------------- */
+typedef struct {
+  void* q_codes;      /* int8 [T_q][H][128], 16-byte aligned */
+  float* q_scale;     /* fp32 [H][ceil(T_q / 128)] */
+  void* k_codes;      /* int8 [T_kv][H][128], logical key order, 16-byte aligned */
+  float* k_scale;     /* fp32 [H][ceil(T_kv / 128)] */
+  float* k_mean;      /* fp32 [H][128], 16-byte aligned */
+  double* k_sum;      /* fp64 [H][128] scratch, 8-byte aligned */
+} wf_qk_i8_t;
+
+/* Byte sizes of the six wf_qk_i8_t buffers, in field order, for a wavefront of num_heads heads.
+ * WF_ERR_SHAPE unless head_dim is 128. */
+int wf_qk_i8_sizes(const wf_wavefront_t* wf, int num_heads, int head_dim, size_t sizes[6]);
+
+/* Quantize q (bf16 [T_q][H][128], the query rows of the wavefront) and the layer's keys (the K
+ * pool through page_table_row, all T_kv tokens) into `qk`.  Errors as wf_attn_forward (a page
+ * outside the pool: WF_ERR_PAGE_OOB from wf_check_status).  Asynchronous on `stream`. */
+int wf_qk_quantize_i8(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* page_table_row,
+                      const wf_wavefront_t* wf, const wf_qk_i8_t* qk, wf_stream_t stream);
+
+/* wf_attn_forward on quantized Q and K (filled by wf_qk_quantize_i8 for the same wavefront and
+ * page table); V is read from kv_pages as in wf_attn_forward.  out, lse_or_null and errors as
+ * wf_attn_forward.  Asynchronous on `stream`. */
+int wf_attn_forward_i8(const wf_qk_i8_t* qk, const wf_kv_pool_t* kv_pages,
+                       const int32_t* page_table_row, const wf_wavefront_t* wf, float scale,
+                       void* out, float* lse_or_null, wf_stream_t stream);
+
+/*
  * Rolling context window: the plan of one round of a stream (host only, no device work).
  *
  * The pages' rules:

@@ -98,7 +98,9 @@ def logits_rows(q_codes, q_scale, k_codes, k_scale, rows: Sequence[int], h: int,
                 softmax_scale: float) -> np.ndarray:
     """fp64 logits [len(rows), n] of query rows `rows` of head h against keys [0, n)."""
     rows = np.asarray(rows)
-    dots = q_codes[rows, h, :].astype(np.int64) @ k_codes[:n, h, :].astype(np.int64).T
+    # |sum| <= 128 * 127^2 < 2^53 and every partial sum is an integer, so the fp64 product is
+    # the exact integer one in any summation order
+    dots = q_codes[rows, h, :].astype(np.float64) @ k_codes[:n, h, :].astype(np.float64).T
     sq = q_scale[h, rows // Q_ROWS].astype(np.float64)[:, None]
     sk = k_scale[h, np.arange(n) // K_KEYS].astype(np.float64)[None, :]
     return softmax_scale * sq * sk * dots.astype(np.float64)
@@ -126,10 +128,14 @@ def attention(q, k, v, chunk_offsets: Sequence[int], num_ctx_chunks: int, softma
                                                         softmax_scale), v64[:off[c + 1], h])
         return out.astype(np.float32)
     out = np.zeros((len(rows), v64.shape[2]), np.float64)
+    rows, heads = np.asarray(rows), np.asarray(heads)
+    # pairs with the same head and the same visible prefix share one matrix product
+    groups = {}
     for i, (r, h) in enumerate(zip(rows, heads)):
-        n = int(kv_end[r])
-        out[i] = _softmax_pv(logits_rows(qc, qs, kc, ks, [r], h, n, softmax_scale),
-                             v64[:n, h])[0]
+        groups.setdefault((int(h), int(kv_end[r])), []).append(i)
+    for (h, n), idx in groups.items():
+        out[idx] = _softmax_pv(logits_rows(qc, qs, kc, ks, rows[idx], h, n, softmax_scale),
+                               v64[:n, h])
     return out.astype(np.float32)
 
 
