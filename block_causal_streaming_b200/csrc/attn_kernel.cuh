@@ -58,9 +58,6 @@
 namespace wfk {
 
 constexpr int kBM = 128;        // query rows per Q tile (UMMA M)
-#ifndef WF_EXP2_POLY_EIGHTHS
-#define WF_EXP2_POLY_EIGHTHS 0   // column pairs out of 8 whose exp2 runs on the FMA pipe
-#endif
 #ifndef WF_KV_RING_KB
 #define WF_KV_RING_KB 160   // K/V ring: 5 tiles of 32 KB at head_dim 128
 #endif
@@ -315,9 +312,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         l *= alpha;
-        // p = exp2(s * scale * log2 e - m2) two columns at a time.  On unmasked tiles
-        // WF_EXP2_POLY_EIGHTHS of every 8 column pairs use the FMA-pipe polynomial and the rest
-        // the MUFU unit.  Masked tiles use the MUFU unit only, so masked columns give exactly 0.
+        // p = exp2(s * scale * log2 e - m2) two columns at a time, every exponential on the
+        // MUFU unit (moving 1/8 or 2/8 of them to an FMA-pipe polynomial measured 3-10 % slower).
         // no visible key yet (possible in a later key split): every p is exactly 0
         const float mref = m2 == -INFINITY ? 0.f : m2;
         const float2 negm = make_float2(-mref, -mref);
@@ -325,36 +321,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // convex combination of the visible values (V = 1 gives exactly 1).
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[BN / 2];
-        // P for column pairs [32 h, 32 h + 32): keys [64 h, 64 h + 64), bf16x2 into TMEM
-        // columns [32 h, 32 h + 32) of S_q.  (Publishing the first half early, so that P.V
-        // starts on it, measured 1-9 % slower.)
-        auto p_half = [&](int h) {
-          if (!masked) {
   #pragma unroll
-            for (int i = 32 * h; i < 32 * h + 32; ++i) {
-              const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2x2, negm);
-              float2 e;
-              if ((i & 7) < WF_EXP2_POLY_EIGHTHS) {
-                e = exp2_poly2(x);
-              } else {
-                e.x = ex2_approx(x.x);
-                e.y = ex2_approx(x.y);
-              }
-              pk[i] = pack_bf16x2(e.x, e.y);
-              acc[i & 3] = add_bf16x2(acc[i & 3], pk[i]);
-            }
-          } else {
+        for (int i = 0; i < BN / 2; ++i) {
+          const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2x2, negm);
+          pk[i] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
+          acc[i & 3] = add_bf16x2(acc[i & 3], pk[i]);
+        }
+        // P into TMEM columns [0, 64) of S_q (bf16 pairs).  (Publishing the first half to the
+        // MMA warp early, so that P.V starts on it, measured 1-9 % slower; storing it early
+        // without publishing it measured no different.)
   #pragma unroll
-            for (int i = 32 * h; i < 32 * h + 32; ++i) {
-              const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2x2, negm);
-              pk[i] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
-              acc[i & 3] = add_bf16x2(acc[i & 3], pk[i]);
-            }
-          }
+        for (int h = 0; h < BN / 64; ++h)
           tmem_st32(tS + 32u * h, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h]));
-        };
-        p_half(0);
-        p_half(1);
         l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
         tmem_wait_st();
         tc_fence_before();

@@ -337,30 +337,5 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
-// Coefficients of a degree-3 polynomial for 2^f on [-1/2, 1/2], fitted for minimal maximum
-// relative error (Lawson's iteratively reweighted least squares on Chebyshev nodes; see
-// exp2_poly.py beside this file).  Maximum relative error 7.5e-5, evaluated in fp32.
-constexpr float kExp2C0 = 0.99992805719375610f;
-constexpr float kExp2C1 = 0.69326096773147583f;
-constexpr float kExp2C2 = 0.24261112511157990f;
-constexpr float kExp2C3 = 0.05517166480422020f;
-
-// 2^x for two values on the FMA pipe instead of the MUFU unit (Cody-Waite style split):
-// x is clamped to >= -126, n = round(x) is formed by adding 1.5 * 2^23 (so n sits in the low
-// mantissa bits), f = x - n lies in [-1/2, 1/2], 2^f comes from the polynomial above, and 2^n is
-// added to the exponent field.  For x >= -126 the exponent never leaves the normal range; below
-// that the result is a tiny positive number instead of the exact underflow to 0.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
-  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-  float2 p = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
-  p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
-  p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
 
 }  // namespace wfk
