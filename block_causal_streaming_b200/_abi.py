@@ -31,7 +31,8 @@ EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror",
             "wf_ipc_export", "wf_ipc_import", "wf_ipc_close", "wf_kv_append_fp8",
             "wf_kv_dequant", "wf_kv_append_publish_fp8", "wf_kv_dequant_published",
             "wf_qk_i8_sizes", "wf_qk_quantize_i8", "wf_attn_forward_i8",
-            "wf_window_slots", "wf_window_round")
+            "wf_attn_forward_segments", "wf_attn_segments_workspace_size",
+            "wf_window_slots", "wf_window_round", "wf_window_round_ring")
 
 
 class WfError(RuntimeError):
@@ -86,7 +87,15 @@ class RoundC(ctypes.Structure):
                 ("num_ctx_chunks", ctypes.c_int32), ("chunk_id", ctypes.c_int64 * 64),
                 ("role", ctypes.c_int32 * 64), ("chunk_stage", ctypes.c_int32 * 64),
                 ("chunk_offsets", ctypes.c_int32 * 65), ("store_to", ctypes.c_int32),
-                ("evicted", ctypes.c_int64)]
+                ("evicted", ctypes.c_int64), ("store_kv_end", ctypes.c_int32)]
+
+
+class SegmentsC(ctypes.Structure):
+    """wf_segments_t."""
+    _fields_ = [("num_segments", ctypes.c_int32),
+                ("rows_end", ctypes.POINTER(ctypes.c_int32)),
+                ("kv_end", ctypes.POINTER(ctypes.c_int32)),
+                ("num_keys", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32)]
 
 
 class Wavefront(ctypes.Structure):
@@ -177,6 +186,17 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wf_window_round.argtypes = [ctypes.POINTER(WindowC), ctypes.c_int64,
                                     ctypes.POINTER(RoundC)]
     lib.wf_window_round.restype = i32
+    lib.wf_window_round_ring.argtypes = [ctypes.POINTER(WindowC), ctypes.c_int64,
+                                         ctypes.POINTER(RoundC)]
+    lib.wf_window_round_ring.restype = i32
+    lib.wf_attn_forward_segments.argtypes = [vp, ctypes.POINTER(KvPool),
+                                             ctypes.POINTER(ctypes.c_int32),
+                                             ctypes.POINTER(SegmentsC), f32, vp,
+                                             ctypes.POINTER(ctypes.c_float), i32, vp,
+                                             ctypes.c_size_t, vp]
+    lib.wf_attn_forward_segments.restype = i32
+    lib.wf_attn_segments_workspace_size.argtypes = [ctypes.POINTER(SegmentsC), i32, i32, i32]
+    lib.wf_attn_segments_workspace_size.restype = ctypes.c_size_t
     return lib
 
 
@@ -293,13 +313,76 @@ def window_slots(window: Window):
     return slots.value, tokens.value
 
 
-def window_round(window: Window, round_index: int) -> RoundC:
-    """wf_window_round: the plan of one round."""
+def window_round(window: Window, round_index: int, ring: bool = False) -> RoundC:
+    """wf_window_round (or, with ring, wf_window_round_ring): the plan of one round."""
     out = RoundC()
-    rc = lib.wf_window_round(ctypes.byref(window.c), int(round_index), ctypes.byref(out))
+    fn = lib.wf_window_round_ring if ring else lib.wf_window_round
+    rc = fn(ctypes.byref(window.c), int(round_index), ctypes.byref(out))
     if rc != WF_OK:
-        raise WfError(rc, "wf_window_round")
+        raise WfError(rc, "wf_window_round_ring" if ring else "wf_window_round")
     return out
+
+
+class Segments:
+    """Host copy of a wf_segments_t; keeps the arrays alive while C reads them."""
+
+    def __init__(self, rows_end: Sequence[int], kv_end: Sequence[int], num_keys: int,
+                 max_pages_per_seq: int):
+        n = len(rows_end)
+        if n != len(kv_end):
+            raise ValueError("rows_end and kv_end need one entry per segment")
+        self._rows = (ctypes.c_int32 * max(n, 1))(*[int(x) for x in rows_end])
+        self._kv = (ctypes.c_int32 * max(n, 1))(*[int(x) for x in kv_end])
+        self.c = SegmentsC(n, ctypes.cast(self._rows, ctypes.POINTER(ctypes.c_int32)),
+                           ctypes.cast(self._kv, ctypes.POINTER(ctypes.c_int32)),
+                           int(num_keys), int(max_pages_per_seq))
+        self.rows_end = [int(x) for x in rows_end]
+        self.kv_end = [int(x) for x in kv_end]
+        self.num_keys = int(num_keys)
+
+    @property
+    def t_q(self) -> int:
+        return self.rows_end[-1] if self.rows_end else 0
+
+
+def attn_segments_workspace_size(seg: Segments, num_heads: int, head_dim: int,
+                                 splits: int = 0) -> int:
+    return int(lib.wf_attn_segments_workspace_size(ctypes.byref(seg.c), int(num_heads),
+                                                   int(head_dim), int(splits)))
+
+
+def attn_forward_segments(q, k_pool, v_pool, page_table_row, seg: Segments, scale: float, out,
+                          lse=None, splits: int = 1, workspace=None, stream=None) -> None:
+    """wf_attn_forward_segments: rows of segment i see logical keys [0, kv_end[i])."""
+    _, page_size, H, D = _pool_shape(k_pool, v_pool)
+    t_q = seg.t_q
+    if tuple(q.shape) != (t_q, H, D) or tuple(out.shape) != (t_q, H, D):
+        raise ValueError(f"q, out: expected [{t_q}, {H}, {D}], got {tuple(q.shape)}, "
+                         f"{tuple(out.shape)}")
+    if lse is not None and tuple(lse.shape) != (H, t_q):
+        raise ValueError(f"lse: expected [{H}, {t_q}], got {tuple(lse.shape)}")
+    if page_table_row.dim() != 1 or page_table_row.numel() < seg.c.max_pages_per_seq:
+        raise ValueError(f"page_table_row: needs {seg.c.max_pages_per_seq} entries")
+    for t, n, d in ((q, "q", "bf16"), (out, "out", "bf16"), (k_pool, "k_pool", "bf16"),
+                    (v_pool, "v_pool", "bf16"), (page_table_row, "page_table_row", "i32")):
+        _check_tensor(t, n, d)
+    if lse is not None:
+        _check_tensor(lse, "lse", "f32")
+    need = attn_segments_workspace_size(seg, H, D, splits)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        raise ValueError(f"workspace: {need} bytes needed for {splits} key splits")
+    pool = _pool_struct(k_pool, v_pool)
+    rc = lib.wf_attn_forward_segments(
+        q.data_ptr(), ctypes.byref(pool),
+        ctypes.cast(ctypes.c_void_p(page_table_row.data_ptr()), ctypes.POINTER(ctypes.c_int32)),
+        ctypes.byref(seg.c), float(scale), out.data_ptr(),
+        ctypes.cast(ctypes.c_void_p(lse.data_ptr()), ctypes.POINTER(ctypes.c_float))
+        if lse is not None else None,
+        int(splits), workspace.data_ptr() if workspace is not None else None,
+        workspace.numel() * workspace.element_size() if workspace is not None else 0,
+        _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_attn_forward_segments")
 
 
 def kv_append(k_pool, v_pool, layer: int, chunk: int, k, v, page_table, wf: WavefrontDesc,

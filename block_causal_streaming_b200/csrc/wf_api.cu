@@ -332,6 +332,35 @@ struct AttnLaunch {
   float* lse_out = nullptr;   // the caller's lse (written by the combine pass when split)
 };
 
+// The query plan of explicit segments: rows [rows_end[i-1], rows_end[i]) see keys [0, kv_end[i]).
+int segments_plan(const wf_segments_t* seg, const wf_kv_pool_t* pool, QueryPlan* qp) {
+  if (seg == nullptr || seg->rows_end == nullptr || seg->kv_end == nullptr)
+    return WF_ERR_INVALID_ARG;
+  if (seg->num_segments < 1 || seg->num_segments > WF_MAX_CHUNKS || seg->num_keys < 1)
+    return WF_ERR_SHAPE;
+  const int64_t pages = (static_cast<int64_t>(seg->num_keys) + pool->page_size - 1) /
+                        pool->page_size;
+  if (seg->max_pages_per_seq < 0 || pages > seg->max_pages_per_seq) return WF_ERR_CAPACITY;
+  qp->nqc = 0;
+  int prev_rows = 0, prev_kv = 1;
+  for (int i = 0; i < seg->num_segments; ++i) {
+    const int r = seg->rows_end[i], n = seg->kv_end[i];
+    if (r < prev_rows) return WF_ERR_SHAPE;                          // rows run forward
+    if (r == prev_rows) continue;                                    // an empty segment
+    if (n < prev_kv || n > seg->num_keys) return WF_ERR_SHAPE;       // limits never decrease
+    qp->row_end[qp->nqc] = r;
+    qp->kv_end[qp->nqc] = n;
+    ++qp->nqc;
+    prev_rows = r;
+    prev_kv = n;
+  }
+  qp->t_q = prev_rows;
+  return WF_OK;
+}
+
+int prepare_common(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* page_table_row,
+                   float scale, void* out, float* lse_or_null, AttnLaunch* L);
+
 int prepare_attention(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* page_table_row,
                       const wf_wavefront_t* wf, float scale, void* out, float* lse_or_null,
                       AttnLaunch* L) {
@@ -341,9 +370,16 @@ int prepare_attention(const void* q, const wf_kv_pool_t* kv_pages, const int32_t
   rc = validate_wavefront(wf, kv_pages, &t_kv);
   if (rc) return rc;
   if (wf->num_ctx_chunks >= wf->num_chunks) return WF_ERR_SHAPE;   // no query chunk
-  if (!(scale > 0.f) || !std::isfinite(scale)) return WF_ERR_INVALID_ARG;
   rc = query_plan(wf, &L->qp);
   if (rc) return rc;
+  return prepare_common(q, kv_pages, page_table_row, scale, out, lse_or_null, L);
+}
+
+// Everything after the query plan: checks of the pointers, tensor maps and kernel parameters.
+int prepare_common(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* page_table_row,
+                   float scale, void* out, float* lse_or_null, AttnLaunch* L) {
+  int rc = WF_OK;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return WF_ERR_INVALID_ARG;
   wfk::AttnParams& p = L->p;
   std::memset(&p, 0, sizeof(p));
   const int t_q = L->qp.t_q;
@@ -540,6 +576,51 @@ int wf_attn_forward_split(const void* q, const wf_kv_pool_t* kv_pages,
     set_split_buffers(&L, S, workspace);
   }
   return launch_attention(&L, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int wf_attn_forward_segments(const void* q, const wf_kv_pool_t* kv_pages,
+                             const int32_t* page_table_row, const wf_segments_t* segments,
+                             float scale, void* out, float* lse_or_null, int splits,
+                             void* workspace, size_t workspace_bytes, wf_stream_t stream) {
+  if (splits < 0) return WF_ERR_INVALID_ARG;
+  int rc = validate_pool(kv_pages);
+  if (rc) return rc;
+  AttnLaunch L;
+  rc = segments_plan(segments, kv_pages, &L.qp);
+  if (rc) return rc;
+  rc = prepare_common(q, kv_pages, page_table_row, scale, out, lse_or_null, &L);
+  if (rc || L.p.T_q == 0) return rc;
+  int S = splits > 0 ? splits : choose_splits(L.qp, L.p.H, L.d->num_sms);
+  S = std::min(S, max_splits(L.qp));
+  if (S > 1) {
+    const size_t need = split_workspace_bytes(L.qp, L.p.H, L.D, S);
+    if (workspace == nullptr || !aligned16(workspace)) return WF_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return WF_ERR_CAPACITY;
+    set_split_buffers(&L, S, workspace);
+  }
+  return launch_attention(&L, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t wf_attn_segments_workspace_size(const wf_segments_t* segments, int num_heads, int head_dim,
+                                       int splits) {
+  QueryPlan qp;
+  wf_kv_pool_t geo{nullptr, nullptr, 1, 16, num_heads, head_dim};
+  if (segments == nullptr || num_heads < 1 || (head_dim != 64 && head_dim != 128) ||
+      splits < 0)
+    return 0;
+  geo.page_size = 16;
+  geo.num_pages = INT32_MAX / 16;
+  wf_segments_t s = *segments;
+  s.max_pages_per_seq = INT32_MAX;          // capacity is checked by the attention call
+  if (segments_plan(&s, &geo, &qp) != WF_OK || qp.t_q == 0) return 0;
+  int S = splits;
+  if (S == 0) {
+    DeviceState* d = nullptr;
+    if (device_state(&d) != WF_OK) return 0;
+    S = choose_splits(qp, num_heads, d->num_sms);
+  }
+  S = std::min(S, max_splits(qp));
+  return split_workspace_bytes(qp, num_heads, head_dim, S);
 }
 
 int wf_attn_forward_split_noalloc(const void* q, const wf_kv_pool_t* kv_pages,

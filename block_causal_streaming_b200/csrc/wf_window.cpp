@@ -84,5 +84,55 @@ int wf_window_round(const wf_window_t* w, int64_t round, wf_round_t* out) {
   out->round = round;
   out->num_chunks = n;
   for (int i = 0; i <= n; ++i) out->chunk_offsets[i] = i * w->chunk_len;
+  // the store pass is the first query chunk: its rows see the slots up to its own
+  out->store_kv_end = -1;
+  for (int i = 0; i < n; ++i)
+    if (out->role[i] == WF_ROLE_STORE) out->store_kv_end = out->chunk_offsets[i + 1];
+  return WF_OK;
+}
+
+int wf_window_round_ring(const wf_window_t* w, int64_t round, wf_round_t* out) {
+  if (out == nullptr) return WF_ERR_INVALID_ARG;
+  const int rc = check_window(w, nullptr, nullptr);
+  if (rc) return rc;
+  if (round < 0) return WF_ERR_INVALID_ARG;
+  const int64_t S = w->num_stages, H = w->history, R = H + 1;   // ring slots
+  const int64_t store = round - S;                 // the chunk in its store pass, if >= 0
+  int n = 0;
+  auto put = [&](int64_t id, int role, int32_t stage) {
+    out->chunk_id[n] = id;
+    out->role[n] = role;
+    out->chunk_stage[n] = stage;
+    ++n;
+  };
+  out->store_to = -1;
+  out->evicted = -1;
+  out->store_kv_end = -1;
+  int ctx = 0;
+  if (store >= 0) {
+    // slot 0: the anchor (chunk 0), in its store pass at round S
+    put(0, store == 0 ? WF_ROLE_STORE : WF_ROLE_ANCHOR, 0);
+    if (store >= 1) {
+      // ring slots 1 .. min(store, R): stored chunks max(1, store - H) .. store, each in slot
+      // 1 + (c - 1) mod R; the slots fill in order, so the occupied ones are contiguous
+      const int64_t occupied = store < R ? store : R;
+      const int64_t first = store - H > 1 ? store - H : 1;
+      for (int64_t slot = 1; slot <= occupied; ++slot) {
+        // the chunk in `slot`: the one in [first, store] congruent to slot - 1 modulo R
+        const int64_t c = first + (((slot - 1) - (first - 1)) % R + R) % R;
+        put(c, c == store ? WF_ROLE_STORE : WF_ROLE_HISTORY, 0);
+      }
+      if (store - R >= 1) out->evicted = store - R;   // its slot now holds the store pass
+    }
+    for (int i = 0; i < n; ++i) ctx += out->role[i] != WF_ROLE_STORE ? 1 : 0;
+  }
+  const int ring_end = n;                           // slots of anchor + occupied ring
+  for (int64_t c = (round - S + 1 > 0 ? round - S + 1 : 0); c <= round; ++c)
+    put(c, WF_ROLE_ACTIVE, w->stages[round - c]);     // in flight, oldest (cleanest) first
+  out->round = round;
+  out->num_chunks = n;
+  out->num_ctx_chunks = ctx;
+  for (int i = 0; i <= n; ++i) out->chunk_offsets[i] = i * w->chunk_len;
+  if (store >= 0) out->store_kv_end = out->chunk_offsets[ring_end];
   return WF_OK;
 }

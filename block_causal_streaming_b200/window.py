@@ -39,6 +39,19 @@ cannot be moved by editing page-table entries.  Nothing that persists is moved, 
 
 :class:`RollingWindow` is the host-side planner: a pure function from the round number to that
 round's descriptor, computed by the library's native planner (``wf_window_round``).
+
+Copy-free form (``copy_free=True``, ``wf_window_round_ring``).  With one GPU per chunk (Wave
+Parallelism), the hand-over append would overwrite a ring slot in the very round in which other
+GPUs may still read the chunk that leaves it.  The copy-free form gives the ring ``history + 1``
+slots instead of ``history`` plus a separate store slot:
+
+    [anchor][ring: ``history + 1`` slots][in flight, cleanest first]
+
+The store pass writes its chunk once, straight into the ring slot it keeps (the slot of the chunk
+that left the history at the end of the previous round), and never moves again.  Its rows see the
+anchor and the whole occupied ring, although their own slot is not the last one, so a round is one
+attention call over query segments (``wf_attn_forward_segments``): the store pass's rows with the
+ring's end as their key limit, then each chunk in flight with its own end.
 :class:`RollingCache` holds the device pools and page tables.  Through the C ABI it runs one
 layer of a round: appends, attention and the hand-over into the ring.
 """
@@ -67,6 +80,7 @@ class RoundView:
     num_ctx_chunks: int         # anchor + history: K/V only, no queries this round
     store_to: Optional[int]     # slot that must also receive the store chunk's K/V after attention
     evicted: Optional[int]      # stream index of the history chunk leaving after this round
+    store_kv_end: Optional[int] = None   # keys the store pass's rows see (None: no store pass)
 
     @property
     def num_chunks(self) -> int:
@@ -82,6 +96,24 @@ class RoundView:
 
     def slot_of(self, chunk_id: int) -> int:
         return self.chunk_ids.index(chunk_id)
+
+    @property
+    def query_rows_slots(self) -> List[int]:
+        """Slots whose chunks carry queries this round, in the order of the query rows: the
+        store pass, then the chunks in flight (slot order in both forms)."""
+        return [i for i, r in enumerate(self.roles) if r in (STORE, ACTIVE)]
+
+    def segments(self):
+        """(rows_end, kv_end) of the round's query segments: one per query chunk, in the order
+        of the query rows; the store pass sees ``store_kv_end`` keys, a chunk in flight the
+        slots up to its own."""
+        rows_end, kv_end, rows = [], [], 0
+        for i in self.query_rows_slots:
+            rows += self.chunk_offsets[i + 1] - self.chunk_offsets[i]
+            rows_end.append(rows)
+            kv_end.append(self.store_kv_end if self.roles[i] == STORE
+                          else self.chunk_offsets[i + 1])
+        return rows_end, kv_end
 
     def rank_view(self, slot: int) -> "RoundView":
         """The call of the one rank whose query chunk is in ``slot`` (Wave Parallelism: one stage,
@@ -105,8 +137,10 @@ class RollingWindow:
     library's native planner; this class only converts it.
     """
 
-    def __init__(self, chunk_len: int, stages: Sequence[int], history: int, page_size: int):
+    def __init__(self, chunk_len: int, stages: Sequence[int], history: int, page_size: int,
+                 copy_free: bool = False):
         from . import _abi
+        self.copy_free = bool(copy_free)
         self.chunk_len = int(chunk_len)
         self.stages = [int(x) for x in stages]
         self.history = int(history)
@@ -121,11 +155,14 @@ class RollingWindow:
                              f"strictly decreasing, at most {MAX_CHUNKS} slots): {e}") from None
         self.pages = math.ceil(self.tokens / self.page_size)
 
+    def slots_and_tokens(self):
+        return self.slots, self.tokens
+
     def view(self, t: int) -> RoundView:
         from . import _abi
         if t < 0:
             raise ValueError("rounds start at 0")
-        r = _abi.window_round(self._w, t)
+        r = _abi.window_round(self._w, t, ring=self.copy_free)
         n = r.num_chunks
         return RoundView(round=int(r.round), chunk_ids=[int(x) for x in r.chunk_id[:n]],
                          roles=[_ROLE_NAMES[x] for x in r.role[:n]],
@@ -133,7 +170,8 @@ class RollingWindow:
                          chunk_offsets=[int(x) for x in r.chunk_offsets[:n + 1]],
                          num_ctx_chunks=int(r.num_ctx_chunks),
                          store_to=None if r.store_to < 0 else int(r.store_to),
-                         evicted=None if r.evicted < 0 else int(r.evicted))
+                         evicted=None if r.evicted < 0 else int(r.evicted),
+                         store_kv_end=None if r.store_kv_end < 0 else int(r.store_kv_end))
 
 
 class RollingCache:
@@ -175,6 +213,9 @@ class RollingCache:
             return
         lay = self.layer_view(view, layer)
         L = self.window.chunk_len
+        if self.window.copy_free:
+            self._run_segments(view, layer, lay, q, k, v, out, scale, lse, stream)
+            return
         for i, slot in enumerate(view.query_slots):
             lay.append(slot, k[i * L:(i + 1) * L], v[i * L:(i + 1) * L], stream)
         lay.forward(q, out, scale=scale, lse=lse, stream=stream)
@@ -182,3 +223,19 @@ class RollingCache:
             # the store chunk is the first query chunk; after this layer's attention the evicted
             # chunk is no longer read, so its slot takes the store chunk's clean K/V
             lay.append(view.store_to, k[:L], v[:L], stream)
+
+    def _run_segments(self, view: RoundView, layer: int, lay, q, k, v, out, scale, lse,
+                      stream) -> None:
+        """Copy-free round: every query chunk is appended once, into its own slot (the store pass
+        into its ring slot), then one attention call over the round's query segments."""
+        from . import _abi
+        L = self.window.chunk_len
+        for i, slot in enumerate(view.query_rows_slots):
+            lay.append(slot, k[i * L:(i + 1) * L], v[i * L:(i + 1) * L], stream)
+        rows_end, kv_end = view.segments()
+        seg = _abi.Segments(rows_end, kv_end, view.chunk_offsets[-1],
+                            self.page_tables.shape[1])
+        if scale is None:
+            scale = 1.0 / math.sqrt(self.pool.head_dim)
+        _abi.attn_forward_segments(q, self.pool.k, self.pool.v, self.page_tables[layer], seg,
+                                   scale, out, lse, 1, None, stream)

@@ -224,6 +224,37 @@ int wf_attn_forward_published(const void* q, const wf_kv_pool_t* kv_pages,
                               void* workspace, size_t workspace_bytes, wf_stream_t stream);
 
 /*
+ * Query segments: attention whose rows carry their own key limit.  Segment i holds query rows
+ * [rows_end[i-1], rows_end[i]) (rows_end[-1] = 0) and sees logical keys [0, kv_end[i]) of the
+ * paged pool; rows_end must not decrease, kv_end must not decrease over the non-empty segments
+ * and lie in [1, num_keys].  The wavefront descriptor is the special case where every query
+ * chunk is a segment whose limit is its own end; segments also express a query chunk that is not
+ * the last of its keys -- the store pass of a copy-free rolling window, whose rows see the whole
+ * history ring although their own slot sits inside it (wf_window_round_ring).
+ */
+typedef struct {
+  int32_t num_segments;        /* 1 .. WF_MAX_CHUNKS */
+  const int32_t* rows_end;     /* host, [num_segments], cumulative query rows */
+  const int32_t* kv_end;       /* host, [num_segments], visible keys of each segment's rows */
+  int32_t num_keys;            /* logical keys the page table maps (>= every kv_end) */
+  int32_t max_pages_per_seq;   /* entries of page_table_row */
+} wf_segments_t;
+
+/*
+ * wf_attn_forward_segments -- wf_attn_forward_split on query segments.  q, out: bf16
+ * [rows_end[last]][H][D]; lse_or_null fp32 [H][rows]; splits, workspace as
+ * wf_attn_forward_split, sized by wf_attn_segments_workspace_size.  WF_ERR_SHAPE for limits that
+ * decrease or exceed num_keys, WF_ERR_CAPACITY when num_keys needs more than max_pages_per_seq
+ * pages; other errors as wf_attn_forward.  Asynchronous on `stream`.
+ */
+int wf_attn_forward_segments(const void* q, const wf_kv_pool_t* kv_pages,
+                             const int32_t* page_table_row, const wf_segments_t* segments,
+                             float scale, void* out, float* lse_or_null, int splits,
+                             void* workspace, size_t workspace_bytes, wf_stream_t stream);
+size_t wf_attn_segments_workspace_size(const wf_segments_t* segments, int num_heads, int head_dim,
+                                       int splits);
+
+/*
  * wf_ipc_export / wf_ipc_import / wf_ipc_close -- share device memory (pools, flag arrays)
  * between processes.  export writes the 64-byte IPC handle of the allocation containing
  * device_ptr (cudaIpcGetMemHandle on its base) and device_ptr's byte offset inside it; import
@@ -413,6 +444,7 @@ typedef struct {
   int32_t chunk_offsets[WF_MAX_CHUNKS + 1];
   int32_t store_to;                            /* slot for the store hand-over, or -1 */
   int64_t evicted;                             /* chunk leaving the history after the round, or -1 */
+  int32_t store_kv_end;                        /* keys the store pass's rows see, or -1 */
 } wf_round_t;
 
 /*
@@ -427,6 +459,22 @@ int wf_window_slots(const wf_window_t* window, int32_t* slots, int64_t* tokens);
  * WF_ERR_INVALID_ARG for a negative round.
  */
 int wf_window_round(const wf_window_t* window, int64_t round, wf_round_t* out);
+
+/*
+ * wf_window_round_ring -- the copy-free plan of round `round`: the same stream, with the history
+ * kept in a ring of history + 1 slots that also holds the store pass.
+ *   [anchor][ring: history + 1 slots][in flight, cleanest first]
+ * The store pass writes its chunk once, straight into the ring slot it keeps as history: the slot
+ * of the chunk that left the history at the end of the previous round (chunk c >= 1 lives in ring
+ * slot 1 + (c - 1) mod (history + 1)).  Nothing is handed over after attention, so no slot is
+ * written in the round in which another GPU may still read it.  The chunks in flight follow the
+ * last occupied ring slot.  Slots are listed in slot order; the store pass's rows see the anchor
+ * and the whole occupied ring (store_kv_end), every chunk in flight sees the slots up to its own.
+ * Query rows run in slot order (store pass first), so the round is one wf_attn_forward_segments
+ * call.  store_to is always -1; num_ctx_chunks counts the anchor and history slots.  Errors as
+ * wf_window_round.
+ */
+int wf_window_round_ring(const wf_window_t* window, int64_t round, wf_round_t* out);
 
 /*
  * wf_check_status -- synchronise `stream`, then return and clear the first error any kernel of

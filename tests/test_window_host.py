@@ -200,3 +200,83 @@ def test_native_planner_argument_checks():
     assert _abi.window_slots(_abi.Window(48, [1000], 61)) == (64, 64 * 48)
     big = _abi.window_round(w, 10 ** 12)                 # far into a stream: 64-bit chunk ids
     assert big.chunk_id[big.num_chunks - 1] == 10 ** 12
+
+
+# ----------------------------------------------------------------- copy-free ring (history + 1)
+def _segment_visible(v, slot):
+    """Chunks whose keys the query chunk in `slot` reads in the round's segment call."""
+    rows_end, kv_end = v.segments()
+    i = v.query_rows_slots.index(slot)
+    n = kv_end[i]
+    return {v.chunk_ids[s] for s in range(v.num_chunks) if v.chunk_offsets[s + 1] <= n}
+
+
+@pytest.mark.parametrize("S,H", SHAPES)
+def test_ring_every_query_chunk_sees_exactly_what_the_pages_name(S, H):
+    win = W.RollingWindow(48, _stages(S), H, 16, copy_free=True)
+    assert (win.slots, win.tokens) == W.RollingWindow(48, _stages(S), H, 16).slots_and_tokens()
+    for t in range(0, 3 * (S + H) + 6):
+        v = win.view(t)
+        assert v.store_to is None                          # nothing is handed over
+        assert v.chunk_offsets == [i * 48 for i in range(v.num_chunks + 1)]
+        assert v.num_chunks <= win.slots and len(set(v.chunk_ids)) == v.num_chunks
+        rows_end, kv_end = v.segments()
+        assert rows_end == [48 * (i + 1) for i in range(len(rows_end))]
+        assert all(a <= b for a, b in zip(kv_end, kv_end[1:]))   # one segment call per round
+        for slot in v.query_rows_slots:
+            c = v.chunk_ids[slot]
+            assert _segment_visible(v, slot) == \
+                expected_visible(t, S, H, c, v.roles[slot] == W.STORE), (t, c)
+
+
+@pytest.mark.parametrize("S,H", SHAPES)
+def test_ring_chunks_are_written_once_and_never_move(S, H):
+    """A stored chunk is written once, by its store pass, straight into the slot it keeps: no
+    round's append ever lands in a slot that holds the anchor or a history chunk."""
+    win = W.RollingWindow(40, _stages(S), H, 16, copy_free=True)
+    home = {}                                              # stored chunk -> its slot
+    for t in range(0, 3 * (S + H) + 6):
+        v = win.view(t)
+        for slot, (c, role) in enumerate(zip(v.chunk_ids, v.roles)):
+            if role in (W.ANCHOR, W.HISTORY):
+                assert home[c] == slot, (t, c)             # where its store pass wrote it
+            if role == W.STORE:
+                assert c not in home
+                written = {s for s in v.query_rows_slots}
+                held = {home[d] for d in v.chunk_ids if d in home}
+                assert slot not in held                    # it overwrites no live history
+                home[c] = slot
+                assert not (written - {slot}) & held       # nor does any other append
+        if v.evicted is not None:
+            assert v.evicted not in v.chunk_ids
+
+
+@pytest.mark.parametrize("S,H,ps", [(2, 2, 16), (3, 1, 32), (1, 3, 16), (4, 0, 48)])
+def test_ring_appends_replayed_with_the_oracle_leave_the_named_chunk_in_every_slot(S, H, ps):
+    """Copy-free: the round's appends (store pass into its ring slot, chunks in flight after the
+    ring), replayed with the oracle's scatter and gather, leave every slot holding the chunk the
+    round names -- stored chunks their store-round rows, with no hand-over."""
+    L, heads, D = 24, 1, 2
+    win = W.RollingWindow(L, _stages(S), H, ps, copy_free=True)
+    rng = np.random.default_rng(4)
+    page_table = rng.permutation(win.pages)
+    pool = np.full((win.pages, ps, heads, D), -1, np.int64)
+    stored = {}
+
+    def rows(c, t):
+        base = (c * 1000 + t) * 100
+        return (base + np.arange(L * heads * D)).reshape(L, heads, D)
+
+    for t in range(0, 3 * (S + H) + 6):
+        v = win.view(t)
+        fresh = {v.chunk_ids[s]: rows(v.chunk_ids[s], t) for s in v.query_rows_slots}
+        for s in v.query_rows_slots:
+            oracle.scatter_chunk(pool, page_table, v.chunk_offsets[s], fresh[v.chunk_ids[s]])
+        logical = oracle.gather_logical(pool, page_table, v.chunk_offsets[-1])
+        for s, c in enumerate(v.chunk_ids):
+            want = fresh[c] if s in v.query_rows_slots else stored[c]
+            assert np.array_equal(logical[v.chunk_offsets[s]:v.chunk_offsets[s + 1]], want), \
+                (t, s, c)
+        if STORE_SLOT(v) is not None:
+            c = v.chunk_ids[STORE_SLOT(v)]
+            stored[c] = fresh[c]
