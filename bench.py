@@ -333,6 +333,52 @@ def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
     return out
 
 
+def int8_leg(wl: Workload, layer, q, dev, stream, steps: int, warmup: int, peak: float,
+             out_bf16) -> dict:
+    """The INT8 attention tier on the workload's layer: wf_qk_quantize_i8 (key mean, int8 codes
+    and scales of K' and Q) and wf_attn_forward_i8, each timed with CUDA events on the launching
+    stream; TFLOP/s on the same algorithmic FLOP count as the bf16 path.  `out_bf16`: the bf16
+    path's output, for the tier's deviation from it."""
+    import block_causal_streaming_b200 as wf
+    from block_causal_streaming_b200.layer import QkI8Buffers
+    qk = QkI8Buffers(layer.desc, wl.heads, wl.head_dim, dev)
+    out = torch.empty_like(q)
+    row = layer.page_tables[layer.layer]
+    scale = 1.0 / np.sqrt(wl.head_dim)
+
+    def quant():
+        wf.qk_quantize_i8(q, layer.pool.k, layer.pool.v, row, layer.desc, qk, stream)
+
+    def attn():
+        wf.attn_forward_i8(qk, layer.pool.k, layer.pool.v, row, layer.desc, scale, out,
+                           None, stream)
+
+    for _ in range(warmup):
+        quant()
+        attn()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for e in evs:
+        e[0].record(stream)
+        quant()
+        e[1].record(stream)
+        attn()
+        e[2].record(stream)
+    torch.cuda.synchronize(dev)
+    rc = wf.check_status()
+    if rc != wf.WF_OK:
+        raise RuntimeError(f"device status after the INT8 leg: {wf.strerror(rc)}")
+    q_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    a_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    flop = attention_flops(wl)
+    dev_abs = (out.float() - out_bf16.float()).abs()
+    return {"steps": steps, "quantize_ms": round(q_ms, 4), "attn_ms": round(a_ms, 4),
+            "attn_tflops": round(flop / (a_ms / 1e3) / 1e12, 2),
+            "frac_of_bf16_peak": round(flop / (a_ms / 1e3) / 1e12 / peak, 4),
+            "vs_bf16_output": {"max_abs": round(float(dev_abs.max()), 5),
+                               "mean_abs": round(float(dev_abs.mean()), 6)}}
+
+
 def gpu_arm(args, world, rank, local):
     import block_causal_streaming_b200 as wf
     from block_causal_streaming_b200.layer import PagedPool, WavefrontLayer
@@ -494,6 +540,14 @@ def gpu_arm(args, world, rank, local):
     if args.fp8_kv:
         res["fp8_kv"] = fp8_kv_leg(wl, layer, k, v, dev, stream, max(5, min(args.steps, 20)),
                                    args.warmup, float(peaks["hbm_gbs"]))
+    if args.int8:
+        if D != 128:
+            res["int8"] = {"unavailable": "the INT8 tier runs head_dim 128"}
+        else:
+            ref_out = torch.empty_like(q)
+            layer.forward(q, ref_out, scale=scale)
+            res["int8"] = int8_leg(wl, layer, q, dev, stream, max(5, min(args.steps, 20)),
+                                   args.warmup, peak, ref_out)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         tflops, info = oracle_sample(wl, inp, target_s=args.cpu_seconds)
         res["cpu_baseline"] = {"value": round(tflops, 6), "unit": UNIT,
@@ -550,6 +604,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--int8", action="store_true",
+                    help="also time the INT8 attention tier (quantize + attention) on the "
+                         "workload's layer")
     ap.add_argument("--fp8-kv", action="store_true",
                     help="also time the FP8 K/V transport kernels (append to e4m3 pages, "
                          "dequantize) on the workload's chunks")
