@@ -23,29 +23,33 @@
 //   warp  9    MMA issuer (one thread): S_q = Q_q K_j^T (SS form) and O_q += P_q V_j (TS form,
 //              P in TMEM)
 //   warps 10-11 idle
-// TMEM (512 columns): S_q at 128 q (128 fp32 columns; P_q, bf16x2, overwrites its first 64) and
-// O_q at 256 + D q.
+// TMEM (512 columns): one S buffer at [0, 128) that the two Q tiles take turns in (128 fp32
+// columns), P_q at [128 + 64 q, 192 + 64 q) (bf16 pairs) and O_q at [256 + D q, 256 + D q + D).
 //
-// Issue order: S_0(0), S_1(0), then for every tile j: P.V_0(j), S_0(j+1), P.V_1(j), S_1(j+1).
-// The two Q tiles run half a period apart: while the softmax of one tile computes P, the tensor
-// pipe works on the other tile's P.V and QK^T, and the two softmax warpgroups do not compete for
-// the exp unit at the same time.  S_q(j+1) overwrites the columns P.V_q(j) reads P from, and is
-// issued right behind it by the same thread without waiting for P.V_q(j) to complete: the tensor
-// core executes one thread's MMAs in issue order, so P.V_q(j) has read its A operand before
-// S_q(j+1) writes those columns.  PTX lists same-accumulator MMA pairs among its pipelined
-// (ordered) pairs; this different-accumulator order is the one NVIDIA's own CUTLASS Blackwell
-// attention mainloop relies on in the same situation (QK^T into S issued straight after the P.V
-// that reads P from S's columns).  Waiting for completion instead cost 4.5 % on the 1.3B 5-step
-// wavefront.
+// Why P has its own columns.  With P written over its own S, QK^T of tile j+1 for a Q tile can
+// only start once P.V of tile j has read P, so every Q tile runs the chain softmax -> P.V ->
+// QK^T -> softmax and the tensor pipe waits on the softmax's whole latency.  TMEM cannot hold two
+// S buffers, two P buffers and two O accumulators at head_dim 128, so the two Q tiles share one
+// S buffer instead: the softmax of a tile hands the buffer back as soon as it has read S into
+// registers, and the next QK^T -- of the other Q tile -- starts then, while the softmax is still
+// computing P.  A QK^T never waits for a P.V.
+//
+// Issue order: S_0(0), S_1(0), then for every tile j >= 1: S_0(j), P.V_0(j-1), S_1(j),
+// P.V_1(j-1), and finally P.V_0(last), P.V_1(last).  S_1(j) waits until softmax 0 has read
+// S_0(j), S_0(j+1) until softmax 1 has read S_1(j); P.V_q(j) waits for P_q(j).  The softmax of
+// tile j writes P_q(j) only after P.V_q(j-1) -- which reads P_q(j-1) from the same columns --
+// has completed; it was issued a tile earlier, so that wait is short.
 //
 // Synchronisation (all mbarriers, all waits bounded):
 //   q_full          TMA -> MMA          Q tiles landed
 //   kv_full[s]      TMA -> MMA          K or V tile landed in slot s
 //   kv_empty[s]     MMA commit -> TMA   slot s free again (both Q tiles' MMAs on it completed)
-//   s_full[q]       MMA commit -> softmax q   S_q of the current tile ready
+//   s_full[q]       MMA commit -> softmax q   S_q of the current tile ready in the S buffer
+//   s_free          softmax -> MMA      the S buffer has been read (one phase per S tile, the
+//                                       two Q tiles alternating; one arrival per warp)
 //   p_full[q]       softmax q -> MMA    P_q written to TMEM (and O_q rescaled if needed)
-//   o_done[q]       MMA commit -> softmax q   P.V_q of the current tile completed (O rescale,
-//                                             epilogue)
+//   o_done[q]       MMA commit -> softmax q   P.V_q of the previous tile completed (P_q free,
+//                                             O rescale, epilogue)
 //   v_zeroed        TMA warp -> MMA     tail rows of the last V tile zeroed
 #pragma once
 
@@ -65,7 +69,7 @@ constexpr int kBN = 128;        // keys per K/V tile (UMMA N of QK^T, K of P.V)
 constexpr int kNQT = 2;         // Q tiles per CTA
 constexpr int kAttnThreads = 384;
 #ifndef WF_REG_SOFTMAX
-#define WF_REG_SOFTMAX 208
+#define WF_REG_SOFTMAX 200
 #endif
 // Register split: the kernel launches with 168 per thread (384 x 168 = 64512); the two softmax
 // warpgroups take kRegSoftmax each and the producer/MMA warpgroup keeps the rest.
@@ -140,6 +144,11 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
+// Positions of K_j and V_j among a unit's 2 nk ring loads, in the order the MMAs use them:
+// K_0, K_1, V_0, K_2, V_1, ..., K_{nk-1}, V_{nk-2}, V_{nk-1}.
+__device__ __forceinline__ int ring_pos_k(int j, int nk) { return j == 0 ? 0 : 2 * j - 1; }
+__device__ __forceinline__ int ring_pos_v(int j, int nk) { return min(2 * j + 2, 2 * nk - 1); }
+
 // kI8: Q and K tiles hold int8 codes (one 128-byte row per query / key at head_dim 128), V
 // stays bf16; the 32 KB Q saves go to a sixth ring slot.
 template <int D, bool kI8 = false>
@@ -158,7 +167,7 @@ struct AttnSmem {
   // barrier indices; per-Q-tile barriers at base + q
   static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NS, B_S = 1 + 2 * NS,
                        B_P = B_S + kNQT, B_O = B_P + kNQT, B_DRAIN = B_O + kNQT,
-                       B_VZ = B_DRAIN + 1, NBAR = B_VZ + 1;
+                       B_VZ = B_DRAIN + 1, B_SF = B_VZ + 1, NBAR = B_SF + 1;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr uint32_t BYTES = MISC_OFF + 16;
   static constexpr uint32_t ALLOC = BYTES + 1024;        // slack for 1024-byte alignment
@@ -210,7 +219,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     *cta_abort = (*reinterpret_cast<volatile unsigned*>(p.grid_abort) == p.launch_id) ? 1 : 0;
     for (int i = 0; i < L::NBAR; ++i)
-      mbar_init(bar(i), (i >= L::B_P && i < L::B_O) ? 128u : 1u);
+      mbar_init(bar(i), (i >= L::B_P && i < L::B_O) ? 128u : i == L::B_SF ? 4u : 1u);
     mbar_init_fence();
   }
   if (warp == 8) {
@@ -233,7 +242,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int row_g = m0 + q * kBM + row;                 // query row
       const int n_r = kv_end_of_row(p, min(row_g, p.T_q - 1));
       const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-      const uint32_t tS = tmem + lane_off + static_cast<uint32_t>(q * 128);
+      const uint32_t tS = tmem + lane_off;                               // the shared S buffer
+      const uint32_t tP = tmem + lane_off + 128u + static_cast<uint32_t>(q * 64);
       const uint32_t tO = tmem + lane_off + 256u + static_cast<uint32_t>(q * D);
       const float sl2 = kI8 ? p.sl2 * __ldg(p.q_scale + head * p.nqt + (m0 + q * kBM) / kBM)
                             : p.sl2;
@@ -254,6 +264,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int c = 0; c < BN / 32; ++c)
             tmem_ld32(tS + 32u * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
           tmem_wait_ld();
+          // S is in registers: the buffer goes to the other Q tile's QK^T (one arrival per warp)
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(L::B_SF));
           if (kI8) {
             // s32 -> fp32, exact: |S| <= 128 x 127^2 < 2^24.  (Reading the bits of
             // 1.5 x 2^23 + S as a float and subtracting 1.5 x 2^23 measured 3 % slower.)
@@ -295,23 +309,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           alpha = ex2_approx(m2 - tmax);                   // 0 on the first visible tile
           m2 = tmax;
         }
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // O_q holds P.V of tiles < j once P.V of tile j-1 has completed; rescale this warp's
-          // rows (threads whose max did not move multiply by 1).
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_O + q), (j - 1) & 1, w));
-          if (!ok) break;
-          tc_fence_after();
-  #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tO + 32u * c, r);
-            tmem_wait_ld();
-  #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(tO + 32u * c, r);
-          }
-        }
-        l *= alpha;
         // p = exp2(s * scale * log2 e - m2) two columns at a time, every exponential on the
         // MUFU unit (moving 1/8 or 2/8 of them to an FMA-pipe polynomial measured 3-10 % slower).
         // no visible key yet (possible in a later key split): every p is exactly 0
@@ -327,13 +324,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           pk[i] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
           acc[i & 3] = add_bf16x2(acc[i & 3], pk[i]);
         }
-        // P into TMEM columns [0, 64) of S_q (bf16 pairs).  (Publishing the first half to the
-        // MMA warp early, so that P.V starts on it, measured 1-9 % slower; storing it early
-        // without publishing it measured no different.)
+        if (j > 0) {
+          // P.V_q(j-1) reads P_q(j-1) from the columns P_q(j) goes to, and O_q holds P.V of the
+          // tiles < j once it has completed (it was issued a tile ago, so this rarely waits).
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_O + q), (j - 1) & 1, w));
+          if (!ok) break;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, need)) {
+            // rescale this warp's rows of O_q (threads whose max did not move multiply by 1)
+  #pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld32(tO + 32u * c, r);
+              tmem_wait_ld();
+  #pragma unroll
+              for (int i = 0; i < 32; ++i)
+                r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+              tmem_st32(tO + 32u * c, r);
+            }
+          }
+        }
+        // P_q into its own 64 TMEM columns (bf16 pairs).
   #pragma unroll
         for (int h = 0; h < BN / 64; ++h)
-          tmem_st32(tS + 32u * h, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h]));
-        l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          tmem_st32(tP + 32u * h, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h]));
+        l = l * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(L::B_P + q));
@@ -410,13 +425,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         return pool_row(p, tok);
       };
       int ready = 0;                                        // chunks known to be published
-      for (int j = 0; j < nk && ok; ++j) {
-        const int coord = box_row(j, lane);                 // lane b resolves box b of tile j
+      // Loads in the order the MMAs use them (ring_pos_k / ring_pos_v): K_0, K_1, V_0, K_2,
+      // V_1, ..., V_{nk-1}.
+      // Lane b holds the pool row of box b of a tile.  Each tile's rows are read from the page
+      // table once, one tile ahead of its K load (the read's latency overlaps the loads in
+      // between), and kept for its V load two loads later.
+      int coord_next = box_row(0, lane);
+      int coord_even = 0, coord_odd = 0;                    // kept for V_j, by the parity of j
+      for (int pos = 0; pos < 2 * nk && ok; ++pos) {
+        const bool last = pos == 2 * nk - 1;
+        const int kv = pos == 0 ? 0 : last ? 1 : (pos & 1) ? 0 : 1;
+        const int j = pos == 0 ? 0 : last ? nk - 1 : (pos & 1) ? (pos + 1) / 2 : (pos - 2) / 2;
+        int coord;
+        if (kv == 0) {
+          coord = coord_next;
+          if (j & 1) coord_odd = coord;
+          else coord_even = coord;
+          if (j + 1 < nk) coord_next = box_row(j + 1, lane);
+        } else {
+          coord = (j & 1) ? coord_odd : coord_even;
+        }
         int cb[BN / 16];
   #pragma unroll
         for (int b = 0; b < BN / 16; ++b) cb[b] = __shfl_sync(0xffffffffu, coord, b);
-        if (kWaitPublished && lane == 0) {
-          // every chunk with a key in this tile must have been published
+        if (kWaitPublished && kv == 0 && lane == 0) {
+          // every chunk with a key in this tile must have been published (K_j is the first
+          // load of tile j)
           const int last_key = min((kb + j + 1) * BN, n_max) - 1;
           const int ready0 = ready;
           while (ok && ready < p.nchunks && (ready == 0 ? 0 : p.chunk_end[ready - 1]) <= last_key) {
@@ -425,32 +459,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           if (ready != ready0) fence_proxy_async_global();
         }
-        if (lane == 0) {
-  #pragma unroll
-          for (int kv = 0; kv < 2 && ok; ++kv) {
-            const int it = 2 * j + kv, slot = it % NS;
-            ok = mbar_wait(bar(L::B_KVE + slot), ((it / NS) & 1) ^ 1, w);
-            if (!ok) break;
+        if (lane == 0 && ok) {
+          const int slot = pos % NS;
+          ok = mbar_wait(bar(L::B_KVE + slot), ((pos / NS) & 1) ^ 1, w);
+          if (ok) {
             const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
             const uint32_t dst = base + L::KV_OFF + slot * KTILE;
             if (kI8 && kv == 0) {
               // int8 K' codes are contiguous in logical key order: one box of BN keys
               mbar_arrive_expect_tx(bar(L::B_KVF + slot), L::KBYTES);
               tma_load_3d(dst, map, 0, head, (kb + j) * BN, bar(L::B_KVF + slot));
-              last_it[slot] = it;
-              continue;
-            }
-            mbar_arrive_expect_tx(bar(L::B_KVF + slot), KTILE);
+            } else {
+              mbar_arrive_expect_tx(bar(L::B_KVF + slot), KTILE);
   #pragma unroll
-            for (int b = 0; b < BN / 16; ++b) {
-              if (b < nb) {
+              for (int b = 0; b < BN / 16; ++b) {
+                if (b < nb) {
   #pragma unroll
-                for (int h = 0; h < DH; ++h)
-                  tma_load_3d(dst + h * KHALF + static_cast<uint32_t>(b * R * 128), map, 64 * h,
-                              head, cb[b], bar(L::B_KVF + slot));
+                  for (int h = 0; h < DH; ++h)
+                    tma_load_3d(dst + h * KHALF + static_cast<uint32_t>(b * R * 128), map,
+                                64 * h, head, cb[b], bar(L::B_KVF + slot));
+                }
               }
             }
-            last_it[slot] = it;
+            last_it[slot] = pos;
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -497,63 +528,116 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool zero_tail = (n_max - (kb + nk - 1) * BN) < BN;   // the loader zeroes V's tail
       bool ok = mbar_wait(bar(L::B_Q), 0, w);
 
-      // S_q(j) = Q_q K_j^T: D/16 K-steps of 16 columns (4 per 128-byte half of a row).
-      auto issue_s_q = [&](int j, int q) {
-        const int slot = (2 * j) % NS;
+      // S(j, q) = Q_q K_j^T into the shared S columns: D/16 K-steps of 16 columns (4 per
+      // 128-byte half of a row; INT8: D/32 steps of 32).  `probe` runs before the last two
+      // steps are issued (see below).
+      constexpr int kStepsS = kI8 ? D / 32 : D / 16, kStepsPV = BN / 16;
+      auto issue_s = [&](int j, int q, auto&& probe) {
+        const int slot = ring_pos_k(j, nk) % NS;
         const uint64_t dk = dk0 + ((static_cast<uint32_t>(slot) * KTILE) >> 4);
-        const uint32_t sd = tmem + static_cast<uint32_t>(q * 128);
         const uint64_t dq = dq0 + ((static_cast<uint32_t>(q) * QTILE) >> 4);
-        if (kI8) {
-          // D int8 values = one 128-byte swizzle row; K-steps of 32 values (32 bytes)
   #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk)
-            umma_ss_i8(sd, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), idesc_qk,
+        for (int kk = 0; kk < kStepsS; ++kk) {
+          if (kk == kStepsS - 2) probe();
+          if (kI8)
+            umma_ss_i8(tmem, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), idesc_qk,
                        kk > 0 ? 1u : 0u);
-        } else {
-  #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ss(sd, dq + (((kk / 4) * QHALF + (kk % 4) * 32) >> 4),
+          else
+            umma_ss(tmem, dq + (((kk / 4) * QHALF + (kk % 4) * 32) >> 4),
                     dk + (((kk / 4) * KHALF + (kk % 4) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(L::B_S + q));
       };
-      auto wait_k = [&](int j) -> bool {
-        const int it = 2 * j;
-        if (!mbar_wait(bar(L::B_KVF + it % NS), (it / NS) & 1, w)) return false;
-        tc_fence_after();
-        return true;
-      };
-      if (ok) ok = wait_k(0);
-      if (ok) {
-        issue_s_q(0, 0);
-        issue_s_q(0, 1);
-        umma_commit(bar(L::B_KVE + 0));
-      }
-      for (int j = 0; ok && j < nk; ++j) {
-        const int itv = 2 * j + 1, slotv = itv % NS;
-        ok = mbar_wait(bar(L::B_KVF + slotv), (itv / NS) & 1, w);
-        if (ok && j == nk - 1 && zero_tail) ok = mbar_wait(bar(L::B_VZ), 0, w);
+      // O_q += P_q(j) V_j, P_q in its own TMEM columns.
+      auto issue_pv = [&](int j, int q, auto&& probe) {
+        const int slotv = ring_pos_v(j, nk) % NS;
         const uint64_t dv = dv0 + ((static_cast<uint32_t>(slotv) * KTILE) >> 4);
-  #pragma unroll 1
-        for (int q = 0; q < kNQT && ok; ++q) {
-          const uint32_t pa = tmem + static_cast<uint32_t>(q * 128);
-          const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
-          ok = mbar_wait(bar(L::B_P + q), j & 1, w);
-          if (!ok) break;
-          tc_fence_after();
+        const uint32_t pa = tmem + 128u + static_cast<uint32_t>(q * 64);
+        const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
   #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            umma_ts(od, pa + 8u * kk, dv + ((kk * 2048u) >> 4), idesc_pv,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(bar(L::B_O + q));
-          if (q == kNQT - 1) umma_commit(bar(L::B_KVE + slotv));   // V_j free
-          if (j + 1 < nk) {
-            if (q == 0) ok = wait_k(j + 1);
-            if (!ok) break;
-            issue_s_q(j + 1, q);            // in issue order behind P.V_q(j), see the header
-            if (q == kNQT - 1) umma_commit(bar(L::B_KVE + (2 * (j + 1)) % NS));   // K_{j+1} free
-          }
+        for (int kk = 0; kk < kStepsPV; ++kk) {
+          if (kk == kStepsPV - 2) probe();
+          umma_ts(od, pa + 8u * kk, dv + ((kk * 2048u) >> 4), idesc_pv,
+                  (j > 0 || kk > 0) ? 1u : 0u);
         }
+        umma_commit(bar(L::B_O + q));
+      };
+      // The tensor pipe takes only a few MMAs ahead of the one executing, so every wait between
+      // two groups of MMAs can leave it idle.  Each group therefore probes the barriers of the
+      // NEXT group (non-blocking) while its last two MMAs are still to be issued and the ones
+      // already queued keep the pipe busy; the blocking wait after the group is skipped when
+      // the probe found them complete.  Barrier state: K_j / V_j landed, the S buffer read
+      // (phase sf, the two Q tiles alternating), P_q(j) written.
+      int sf = 0;             // S-free phases consumed: one per S tile read by a softmax
+      bool ready = false;     // the next group's barriers are known to be complete
+      auto kv_done = [&](int pos) { return mbar_test(bar(L::B_KVF + pos % NS), (pos / NS) & 1); };
+      auto wait_kv = [&](int pos) -> bool {
+        return mbar_wait(bar(L::B_KVF + pos % NS), (pos / NS) & 1, w);
+      };
+      auto s_free_done = [&]() { return mbar_test(bar(L::B_SF), sf & 1); };
+      auto wait_s_free = [&]() -> bool { return mbar_wait(bar(L::B_SF), sf & 1, w); };
+      auto p_done = [&](int j, int q) { return mbar_test(bar(L::B_P + q), j & 1); };
+      auto wait_p = [&](int j, int q) -> bool { return mbar_wait(bar(L::B_P + q), j & 1, w); };
+      // what PV(j, 0) needs: V_j (tail rows zeroed for the last tile) and P_0(j)
+      auto pv0_done = [&](int j) {
+        return kv_done(ring_pos_v(j, nk)) &&
+               (j < nk - 1 || !zero_tail || mbar_test(bar(L::B_VZ), 0)) && p_done(j, 0);
+      };
+      auto wait_pv0 = [&](int j) -> bool {
+        return wait_kv(ring_pos_v(j, nk)) &&
+               (j < nk - 1 || !zero_tail || mbar_wait(bar(L::B_VZ), 0, w)) && wait_p(j, 0);
+      };
+      auto no_probe = [] {};
+      if (ok) ok = wait_kv(0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0, no_probe);
+        ok = wait_s_free();
+      }
+      if (ok) {
+        ++sf;
+        tc_fence_after();
+        issue_s(0, 1, no_probe);
+        umma_commit(bar(L::B_KVE + ring_pos_k(0, nk) % NS));   // K_0 free
+      }
+      if (ok && nk > 1) ok = wait_kv(ring_pos_k(1, nk)) && wait_s_free();
+      for (int j = 1; ok && j < nk; ++j) {
+        // S(j, 0): K_j landed and softmax 1 has read S_1(j-1) (checked above)
+        ++sf;
+        tc_fence_after();
+        issue_s(j, 0, [&] { ready = pv0_done(j - 1); });
+        if (!ready) ok = wait_pv0(j - 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(j - 1, 0, [&] { ready = s_free_done(); });
+        if (!ready) ok = wait_s_free();
+        if (!ok) break;
+        ++sf;
+        tc_fence_after();
+        issue_s(j, 1, [&] { ready = p_done(j - 1, 1); });
+        umma_commit(bar(L::B_KVE + ring_pos_k(j, nk) % NS));   // K_j free
+        if (!ready) ok = wait_p(j - 1, 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (j + 1 < nk) {
+          issue_pv(j - 1, 1, [&] { ready = kv_done(ring_pos_k(j + 1, nk)) && s_free_done(); });
+          umma_commit(bar(L::B_KVE + ring_pos_v(j - 1, nk) % NS));   // V_{j-1} free
+          if (!ready) ok = wait_kv(ring_pos_k(j + 1, nk)) && wait_s_free();
+        } else {
+          issue_pv(j - 1, 1, no_probe);
+          umma_commit(bar(L::B_KVE + ring_pos_v(j - 1, nk) % NS));   // V_{j-1} free
+        }
+      }
+      if (ok) ok = wait_pv0(nk - 1);
+      if (ok) {
+        tc_fence_after();
+        issue_pv(nk - 1, 0, no_probe);
+        ok = wait_p(nk - 1, 1);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_pv(nk - 1, 1, no_probe);
+        umma_commit(bar(L::B_KVE + ring_pos_v(nk - 1, nk) % NS));   // V_{nk-1} free
       }
       // every MMA this thread issued must complete before TMEM is released
       umma_commit(bar(L::B_DRAIN));
