@@ -17,12 +17,12 @@
 // Warp roles (384 threads):
 //   warps 0-3  softmax of Q tile 0: thread t owns query row t (TMEM lane t)
 //   warps 4-7  softmax of Q tile 1
-//   warp  8    TMA producer: Q tiles once, then K_j, V_j (128 keys each) into a ring of NS
-//              shared-memory slots, page by page through the page table; zeroes the rows of
-//              the last V tile past the last visible key; allocates/frees TMEM
-//   warp  9    MMA issuer (one thread): S_q = Q_q K_j^T (SS form) and O_q += P_q V_j (TS form,
-//              P in TMEM)
-//   warps 10-11 idle
+//   warp  8    TMA producer of Q (once) and of K_j (128 keys each) into the K ring, page by page
+//              through the page table; allocates/frees TMEM
+//   warp 11    TMA producer of V_j into the V ring; zeroes the rows of the last V tile past
+//              the last visible key
+//   warp  9    QK^T issuer (one thread): S_q = Q_q K_j^T (SS form)
+//   warp 10    P.V issuer (one thread): O_q += P_q V_j (TS form, P in TMEM)
 // TMEM (512 columns): one S buffer at [0, 128) that the two Q tiles take turns in (128 fp32
 // columns), P_q at [128 + 64 q, 192 + 64 q) (bf16 pairs) and O_q at [256 + D q, 256 + D q + D).
 //
@@ -34,16 +34,17 @@
 // registers, and the next QK^T -- of the other Q tile -- starts then, while the softmax is still
 // computing P.  A QK^T never waits for a P.V.
 //
-// Issue order: S_0(0), S_1(0), then for every tile j >= 1: S_0(j), P.V_0(j-1), S_1(j),
-// P.V_1(j-1), and finally P.V_0(last), P.V_1(last).  S_1(j) waits until softmax 0 has read
-// S_0(j), S_0(j+1) until softmax 1 has read S_1(j); P.V_q(j) waits for P_q(j).  The softmax of
-// tile j writes P_q(j) only after P.V_q(j-1) -- which reads P_q(j-1) from the same columns --
-// has completed; it was issued a tile earlier, so that wait is short.
+// Issue order: the QK^T thread issues S_0(0), S_1(0), S_0(1), S_1(1), ...; S_1(j) waits until
+// softmax 0 has read S_0(j), S_0(j+1) until softmax 1 has read S_1(j).  The P.V thread issues
+// P.V_0(0), P.V_1(0), P.V_0(1), ...; P.V_q(j) waits for P_q(j).  The softmax of tile j writes
+// P_q(j) only after P.V_q(j-1) -- which reads P_q(j-1) from the same columns -- has completed;
+// it was issued a tile earlier, so that wait is short.
 //
 // Synchronisation (all mbarriers, all waits bounded):
 //   q_full          TMA -> MMA          Q tiles landed
 //   kv_full[s]      TMA -> MMA          K or V tile landed in slot s
-//   kv_empty[s]     MMA commit -> TMA   slot s free again (both Q tiles' MMAs on it completed)
+//   kv_empty[s]     MMA commit -> TMA   slot s free again (both Q tiles' MMAs on it completed;
+//                                       K slots freed by the QK^T thread, V slots by the P.V one)
 //   s_full[q]       MMA commit -> softmax q   S_q of the current tile ready in the S buffer
 //   s_free          softmax -> MMA      the S buffer has been read (one phase per S tile, the
 //                                       two Q tiles alternating; one arrival per warp)
@@ -68,6 +69,9 @@ constexpr int kBM = 128;        // query rows per Q tile (UMMA M)
 constexpr int kBN = 128;        // keys per K/V tile (UMMA N of QK^T, K of P.V)
 constexpr int kNQT = 2;         // Q tiles per CTA
 constexpr int kAttnThreads = 384;
+#ifndef WF_K_SLOTS
+#define WF_K_SLOTS 0      // K slots of the K/V ring; 0: half of the slots, rounded down
+#endif
 #ifndef WF_REG_SOFTMAX
 #define WF_REG_SOFTMAX 200
 #endif
@@ -144,11 +148,6 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-// Positions of K_j and V_j among a unit's 2 nk ring loads, in the order the MMAs use them:
-// K_0, K_1, V_0, K_2, V_1, ..., K_{nk-1}, V_{nk-2}, V_{nk-1}.
-__device__ __forceinline__ int ring_pos_k(int j, int nk) { return j == 0 ? 0 : 2 * j - 1; }
-__device__ __forceinline__ int ring_pos_v(int j, int nk) { return min(2 * j + 2, 2 * nk - 1); }
-
 // kI8: Q and K tiles hold int8 codes (one 128-byte row per query / key at head_dim 128), V
 // stays bf16; the 32 KB Q saves go to a sixth ring slot.
 template <int D, bool kI8 = false>
@@ -156,6 +155,10 @@ struct AttnSmem {
   static constexpr int BN = kBN;
   static constexpr int DH = D / 64;                      // 128-byte halves of a bf16 row
   static constexpr int NS = (WF_KV_RING_KB + (kI8 ? 32 : 0)) * 1024 / (int)(DH * BN * 128);
+  // Slots [0, NSK) hold K tiles, [NSK, NS) V tiles: two rings, each filled by its own producer
+  // warp, so K loads never wait behind V tiles that the later P.V still holds.
+  static constexpr int NSK = WF_K_SLOTS > 0 ? WF_K_SLOTS : NS / 2, NSV = NS - NSK;
+  static_assert(NSK >= 1 && NSV >= 1, "each ring needs a slot");
   static constexpr uint32_t QHALF = kBM * 128u;          // 128 rows x 128 B, 128B-swizzled
   static constexpr uint32_t QTILE = kI8 ? QHALF : DH * QHALF;
   static constexpr uint32_t KBYTES = kI8 ? BN * 128u : DH * BN * 128u;   // bytes a K tile loads
@@ -167,7 +170,7 @@ struct AttnSmem {
   // barrier indices; per-Q-tile barriers at base + q
   static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NS, B_S = 1 + 2 * NS,
                        B_P = B_S + kNQT, B_O = B_P + kNQT, B_DRAIN = B_O + kNQT,
-                       B_VZ = B_DRAIN + 1, B_SF = B_VZ + 1, NBAR = B_SF + 1;
+                       B_VZ = B_DRAIN + 2, B_SF = B_VZ + 1, NBAR = B_SF + 1;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr uint32_t BYTES = MISC_OFF + 16;
   static constexpr uint32_t ALLOC = BYTES + 1024;        // slack for 1024-byte alignment
@@ -399,17 +402,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegOther) : "memory");
-    if (!skip && warp == 8) {
-      // ------------------------------------------------------------------------ TMA producer
+    if (!skip && (warp == 8 || warp == 11)) {
+      // ------------------------------------------------------------------------ TMA producers
+      // Warp 8 loads the Q tiles, then K_0, K_1, ... into the K ring; warp 11 loads V_0, V_1,
+      // ... into the V ring and zeroes the rows of the last V tile past the last visible key.
+      const int kv = warp == 8 ? 0 : 1;
+      const int ns = kv ? L::NSV : L::NSK, s0 = kv ? L::NSK : 0;
       const int R = p.box_rows, nb = BN / R;             // page boxes per K/V tile (<= BN/16)
       bool ok = true;
-      int last_it[NS];
-  #pragma unroll
-      for (int s = 0; s < NS; ++s) last_it[s] = -1;
-      if (lane == 0) {
+      if (kv == 0 && lane == 0) {
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_k);
-        tma_prefetch_desc(&p.tm_v);
         mbar_arrive_expect_tx(bar(L::B_Q), kNQT * QTILE);
   #pragma unroll
         for (int qt = 0; qt < kNQT; ++qt)
@@ -418,6 +421,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tma_load_3d(base + L::Q_OFF + qt * QTILE + h * QHALF, &p.tm_q, 64 * h, head,
                         m0 + qt * kBM, bar(L::B_Q));
       }
+      if (kv == 1 && lane == 0) tma_prefetch_desc(&p.tm_v);
+      const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
       // Physical row of box b of tile t (past the pool -- TMA fills zeros -- beyond n_max).
       auto box_row = [&](int t, int b) -> int {
         const int tok = (kb + t) * BN + b * R;
@@ -425,32 +430,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         return pool_row(p, tok);
       };
       int ready = 0;                                        // chunks known to be published
-      // Loads in the order the MMAs use them (ring_pos_k / ring_pos_v): K_0, K_1, V_0, K_2,
-      // V_1, ..., V_{nk-1}.
-      // Lane b holds the pool row of box b of a tile.  Each tile's rows are read from the page
-      // table once, one tile ahead of its K load (the read's latency overlaps the loads in
-      // between), and kept for its V load two loads later.
+      int issued = 0;                                       // tiles whose loads were issued
+      // Lane b holds the pool row of box b of a tile, read from the page table one tile ahead
+      // so that the read's latency overlaps the load before it.
       int coord_next = box_row(0, lane);
-      int coord_even = 0, coord_odd = 0;                    // kept for V_j, by the parity of j
-      for (int pos = 0; pos < 2 * nk && ok; ++pos) {
-        const bool last = pos == 2 * nk - 1;
-        const int kv = pos == 0 ? 0 : last ? 1 : (pos & 1) ? 0 : 1;
-        const int j = pos == 0 ? 0 : last ? nk - 1 : (pos & 1) ? (pos + 1) / 2 : (pos - 2) / 2;
-        int coord;
-        if (kv == 0) {
-          coord = coord_next;
-          if (j & 1) coord_odd = coord;
-          else coord_even = coord;
-          if (j + 1 < nk) coord_next = box_row(j + 1, lane);
-        } else {
-          coord = (j & 1) ? coord_odd : coord_even;
-        }
+      for (int j = 0; j < nk && ok; ++j) {
+        const int coord = coord_next;
+        if (j + 1 < nk) coord_next = box_row(j + 1, lane);
         int cb[BN / 16];
   #pragma unroll
         for (int b = 0; b < BN / 16; ++b) cb[b] = __shfl_sync(0xffffffffu, coord, b);
-        if (kWaitPublished && kv == 0 && lane == 0) {
-          // every chunk with a key in this tile must have been published (K_j is the first
-          // load of tile j)
+        if (kWaitPublished && lane == 0) {
+          // every chunk with a key in this tile must have been published
           const int last_key = min((kb + j + 1) * BN, n_max) - 1;
           const int ready0 = ready;
           while (ok && ready < p.nchunks && (ready == 0 ? 0 : p.chunk_end[ready - 1]) <= last_key) {
@@ -460,10 +451,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (ready != ready0) fence_proxy_async_global();
         }
         if (lane == 0 && ok) {
-          const int slot = pos % NS;
-          ok = mbar_wait(bar(L::B_KVE + slot), ((pos / NS) & 1) ^ 1, w);
+          const int slot = s0 + j % ns;
+          ok = mbar_wait(bar(L::B_KVE + slot), ((j / ns) & 1) ^ 1, w);
           if (ok) {
-            const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
             const uint32_t dst = base + L::KV_OFF + slot * KTILE;
             if (kI8 && kv == 0) {
               // int8 K' codes are contiguous in logical key order: one box of BN keys
@@ -481,17 +471,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
               }
             }
-            last_it[slot] = pos;
+            issued = j + 1;
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
       }
       const int zero_from = n_max - (kb + nk - 1) * BN;    // rows >= this of the last V tile
-      if (ok && zero_from < BN) {
+      if (kv == 1 && ok && zero_from < BN) {
         // Rows past the last visible key may hold anything (even NaN, which 0 * NaN would spread
-        // through P.V); once the last V tile has landed, zero them and release the MMA warp.
-        const int it = 2 * (nk - 1) + 1, slot = it % NS;
-        if (lane == 0) ok = mbar_wait(bar(L::B_KVF + slot), (it / NS) & 1, w);
+        // through P.V); once the last V tile has landed, zero them and release the P.V thread.
+        const int slot = s0 + (nk - 1) % ns;
+        if (lane == 0) ok = mbar_wait(bar(L::B_KVF + slot), ((nk - 1) / ns) & 1, w);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (ok) {
           const uint32_t vb = base + L::KV_OFF + slot * KTILE;
@@ -507,141 +497,98 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       if (lane == 0) {
-        // every load this warp issued must land before shared memory is released
-        mbar_wait_drain(bar(L::B_Q), 0);
-  #pragma unroll
-        for (int s = 0; s < NS; ++s)
-          if (last_it[s] >= 0) mbar_wait_drain(bar(L::B_KVF + s), (last_it[s] / NS) & 1);
+        // every load this warp issued must land before shared memory is released: the last
+        // issued tile of each slot (tiles were loaded in order)
+        if (kv == 0) mbar_wait_drain(bar(L::B_Q), 0);
+        for (int r = 0; r < ns && r < issued; ++r) {
+          const int jl = issued - 1 - ((issued - 1 - r) % ns);   // last tile in slot s0 + r
+          mbar_wait_drain(bar(L::B_KVF + s0 + jl % ns), (jl / ns) & 1);
+        }
       }
-    } else if (!skip && warp == 9 && lane == 0) {
-      // ---------------------------------------------------------------------- MMA issuer
-      // One thread issues everything in a fixed order.  Descriptors are built once; per
-      // instruction only a compile-time offset (16-byte units) is added to the start-address
-      // field, so one MMA costs a few instructions to issue -- the tensor core retires a
-      // 128 x BN x 16 step in BN/2 cycles and must not wait for the issuer.
+    } else if (!skip && (warp == 9 || warp == 10) && lane == 0) {
+      // ---------------------------------------------------------------------- MMA issuers
+      // Two threads: warp 9 issues every QK^T, warp 10 every P.V.  A chain of MMAs into one
+      // accumulator issued by one thread runs at about 88 cycles per 128 x 128 x 16 step for
+      // QK^T (operands in SMEM) and 128 for P.V (P from TMEM), against 64 at the tensor core's
+      // rate; two independent chains in flight together run at the full rate.  Descriptors are
+      // built once; per instruction only a compile-time offset (16-byte units) is added to the
+      // start-address field, so the issue loop stays a few instructions per MMA.
       constexpr uint32_t idesc_qk = kI8 ? idesc_s8_s32(kBM, BN)      // Q, K both K-major
                                         : idesc_bf16_f32(kBM, BN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);     // P (TMEM), V MN-major
       const uint64_t dq0 = smem_desc_sw128(base + L::Q_OFF, 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(base + L::KV_OFF, 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(base + L::KV_OFF, KHALF, 1024);
-      const bool zero_tail = (n_max - (kb + nk - 1) * BN) < BN;   // the loader zeroes V's tail
-      bool ok = mbar_wait(bar(L::B_Q), 0, w);
-
-      // S(j, q) = Q_q K_j^T into the shared S columns: D/16 K-steps of 16 columns (4 per
-      // 128-byte half of a row; INT8: D/32 steps of 32).  `probe` runs before the last two
-      // steps are issued (see below).
-      constexpr int kStepsS = kI8 ? D / 32 : D / 16, kStepsPV = BN / 16;
-      auto issue_s = [&](int j, int q, auto&& probe) {
-        const int slot = ring_pos_k(j, nk) % NS;
-        const uint64_t dk = dk0 + ((static_cast<uint32_t>(slot) * KTILE) >> 4);
-        const uint64_t dq = dq0 + ((static_cast<uint32_t>(q) * QTILE) >> 4);
+      bool ok = true;
+      constexpr int NSK = L::NSK, NSV = L::NSV;
+      if (warp == 9) {
+        // S(j, q) = Q_q K_j^T into the shared S columns: D/16 K-steps of 16 columns (4 per
+        // 128-byte half of a row; INT8: D/32 steps of 32).  S(j, 0) waits for K_j and, after
+        // the first tile, for softmax 1 to have read S_1(j-1); S(j, 1) for softmax 0 to have
+        // read S_0(j).
+        constexpr int kSteps = kI8 ? D / 32 : D / 16;
+        auto issue_s = [&](int j, int q) {
+          const int slot = j % NSK;
+          const uint64_t dk = dk0 + ((static_cast<uint32_t>(slot) * KTILE) >> 4);
+          const uint64_t dq = dq0 + ((static_cast<uint32_t>(q) * QTILE) >> 4);
   #pragma unroll
-        for (int kk = 0; kk < kStepsS; ++kk) {
-          if (kk == kStepsS - 2) probe();
-          if (kI8)
-            umma_ss_i8(tmem, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), idesc_qk,
-                       kk > 0 ? 1u : 0u);
-          else
-            umma_ss(tmem, dq + (((kk / 4) * QHALF + (kk % 4) * 32) >> 4),
-                    dk + (((kk / 4) * KHALF + (kk % 4) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kSteps; ++kk) {
+            if (kI8)
+              umma_ss_i8(tmem, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), idesc_qk,
+                         kk > 0 ? 1u : 0u);
+            else
+              umma_ss(tmem, dq + (((kk / 4) * QHALF + (kk % 4) * 32) >> 4),
+                      dk + (((kk / 4) * KHALF + (kk % 4) * 32) >> 4), idesc_qk,
+                      kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar(L::B_S + q));
+        };
+        int sf = 0;           // S-free phases consumed: one per S tile read by a softmax
+        ok = mbar_wait(bar(L::B_Q), 0, w);
+        for (int j = 0; ok && j < nk; ++j) {
+          ok = mbar_wait(bar(L::B_KVF + j % NSK), (j / NSK) & 1, w);
+          if (ok && j > 0) ok = mbar_wait(bar(L::B_SF), (sf++) & 1, w);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(j, 0);
+          ok = mbar_wait(bar(L::B_SF), (sf++) & 1, w);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(j, 1);
+          umma_commit(bar(L::B_KVE + j % NSK));                  // K_j free
         }
-        umma_commit(bar(L::B_S + q));
-      };
-      // O_q += P_q(j) V_j, P_q in its own TMEM columns.
-      auto issue_pv = [&](int j, int q, auto&& probe) {
-        const int slotv = ring_pos_v(j, nk) % NS;
-        const uint64_t dv = dv0 + ((static_cast<uint32_t>(slotv) * KTILE) >> 4);
-        const uint32_t pa = tmem + 128u + static_cast<uint32_t>(q * 64);
-        const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
+      } else {
+        // PV(j, q): O_q += P_q(j) V_j (BN/16 K-steps, P_q in its own TMEM columns), once V_j
+        // has landed (tail rows zeroed for the last tile) and P_q(j) is written.
+        const bool zero_tail = (n_max - (kb + nk - 1) * BN) < BN;   // the loader zeroes V's tail
+        auto issue_pv = [&](int j, int q) {
+          const int slotv = NSK + j % NSV;
+          const uint64_t dv = dv0 + ((static_cast<uint32_t>(slotv) * KTILE) >> 4);
+          const uint32_t pa = tmem + 128u + static_cast<uint32_t>(q * 64);
+          const uint32_t od = tmem + 256u + static_cast<uint32_t>(q * D);
   #pragma unroll
-        for (int kk = 0; kk < kStepsPV; ++kk) {
-          if (kk == kStepsPV - 2) probe();
-          umma_ts(od, pa + 8u * kk, dv + ((kk * 2048u) >> 4), idesc_pv,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_ts(od, pa + 8u * kk, dv + ((kk * 2048u) >> 4), idesc_pv,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar(L::B_O + q));
+        };
+        for (int j = 0; ok && j < nk; ++j) {
+          ok = mbar_wait(bar(L::B_KVF + NSK + j % NSV), (j / NSV) & 1, w);
+          if (ok && j == nk - 1 && zero_tail) ok = mbar_wait(bar(L::B_VZ), 0, w);
+          if (ok) ok = mbar_wait(bar(L::B_P + 0), j & 1, w);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(j, 0);
+          ok = mbar_wait(bar(L::B_P + 1), j & 1, w);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(j, 1);
+          umma_commit(bar(L::B_KVE + NSK + j % NSV));            // V_j free
         }
-        umma_commit(bar(L::B_O + q));
-      };
-      // The tensor pipe takes only a few MMAs ahead of the one executing, so every wait between
-      // two groups of MMAs can leave it idle.  Each group therefore probes the barriers of the
-      // NEXT group (non-blocking) while its last two MMAs are still to be issued and the ones
-      // already queued keep the pipe busy; the blocking wait after the group is skipped when
-      // the probe found them complete.  Barrier state: K_j / V_j landed, the S buffer read
-      // (phase sf, the two Q tiles alternating), P_q(j) written.
-      int sf = 0;             // S-free phases consumed: one per S tile read by a softmax
-      bool ready = false;     // the next group's barriers are known to be complete
-      auto kv_done = [&](int pos) { return mbar_test(bar(L::B_KVF + pos % NS), (pos / NS) & 1); };
-      auto wait_kv = [&](int pos) -> bool {
-        return mbar_wait(bar(L::B_KVF + pos % NS), (pos / NS) & 1, w);
-      };
-      auto s_free_done = [&]() { return mbar_test(bar(L::B_SF), sf & 1); };
-      auto wait_s_free = [&]() -> bool { return mbar_wait(bar(L::B_SF), sf & 1, w); };
-      auto p_done = [&](int j, int q) { return mbar_test(bar(L::B_P + q), j & 1); };
-      auto wait_p = [&](int j, int q) -> bool { return mbar_wait(bar(L::B_P + q), j & 1, w); };
-      // what PV(j, 0) needs: V_j (tail rows zeroed for the last tile) and P_0(j)
-      auto pv0_done = [&](int j) {
-        return kv_done(ring_pos_v(j, nk)) &&
-               (j < nk - 1 || !zero_tail || mbar_test(bar(L::B_VZ), 0)) && p_done(j, 0);
-      };
-      auto wait_pv0 = [&](int j) -> bool {
-        return wait_kv(ring_pos_v(j, nk)) &&
-               (j < nk - 1 || !zero_tail || mbar_wait(bar(L::B_VZ), 0, w)) && wait_p(j, 0);
-      };
-      auto no_probe = [] {};
-      if (ok) ok = wait_kv(0);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0, no_probe);
-        ok = wait_s_free();
-      }
-      if (ok) {
-        ++sf;
-        tc_fence_after();
-        issue_s(0, 1, no_probe);
-        umma_commit(bar(L::B_KVE + ring_pos_k(0, nk) % NS));   // K_0 free
-      }
-      if (ok && nk > 1) ok = wait_kv(ring_pos_k(1, nk)) && wait_s_free();
-      for (int j = 1; ok && j < nk; ++j) {
-        // S(j, 0): K_j landed and softmax 1 has read S_1(j-1) (checked above)
-        ++sf;
-        tc_fence_after();
-        issue_s(j, 0, [&] { ready = pv0_done(j - 1); });
-        if (!ready) ok = wait_pv0(j - 1);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(j - 1, 0, [&] { ready = s_free_done(); });
-        if (!ready) ok = wait_s_free();
-        if (!ok) break;
-        ++sf;
-        tc_fence_after();
-        issue_s(j, 1, [&] { ready = p_done(j - 1, 1); });
-        umma_commit(bar(L::B_KVE + ring_pos_k(j, nk) % NS));   // K_j free
-        if (!ready) ok = wait_p(j - 1, 1);
-        if (!ok) break;
-        tc_fence_after();
-        if (j + 1 < nk) {
-          issue_pv(j - 1, 1, [&] { ready = kv_done(ring_pos_k(j + 1, nk)) && s_free_done(); });
-          umma_commit(bar(L::B_KVE + ring_pos_v(j - 1, nk) % NS));   // V_{j-1} free
-          if (!ready) ok = wait_kv(ring_pos_k(j + 1, nk)) && wait_s_free();
-        } else {
-          issue_pv(j - 1, 1, no_probe);
-          umma_commit(bar(L::B_KVE + ring_pos_v(j - 1, nk) % NS));   // V_{j-1} free
-        }
-      }
-      if (ok) ok = wait_pv0(nk - 1);
-      if (ok) {
-        tc_fence_after();
-        issue_pv(nk - 1, 0, no_probe);
-        ok = wait_p(nk - 1, 1);
-      }
-      if (ok) {
-        tc_fence_after();
-        issue_pv(nk - 1, 1, no_probe);
-        umma_commit(bar(L::B_KVE + ring_pos_v(nk - 1, nk) % NS));   // V_{nk-1} free
       }
       // every MMA this thread issued must complete before TMEM is released
-      umma_commit(bar(L::B_DRAIN));
-      mbar_wait_drain(bar(L::B_DRAIN), 0);
+      umma_commit(bar(L::B_DRAIN + (warp - 9)));
+      mbar_wait_drain(bar(L::B_DRAIN + (warp - 9)), 0);
     }
   }
 
