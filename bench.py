@@ -267,10 +267,12 @@ def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
                hbm_peak: float) -> dict:
     """The FP8 transport kernels over every chunk of the workload's layer: wf_kv_append_fp8
     (bf16 rows -> e4m3 pages + per-(token, head) scales) and wf_kv_dequant (back into the bf16
-    pool), each leg timed with CUDA events on the launching stream after a 256 MB read that
-    evicts L2.  The read writes back whatever the previous leg left dirty, outside the timed
-    region, and leaves L2 holding clean lines only.  Algorithmic bytes: every K/V element read
-    once in one format and written once in the other."""
+    pool), one launch per chunk as a Wave-Parallelism producer and consumer run them, and the
+    chunk-range forms (wf_kv_append_fp8_chunks / wf_kv_dequant_chunks) over the whole layer in
+    one launch each.  Each leg is timed with CUDA events on the launching stream after a 256 MB
+    read that evicts L2; the read writes back whatever the previous leg left dirty, outside the
+    timed region, and leaves L2 holding clean lines only.  Algorithmic bytes: every K/V element
+    read once in one format and written once in the other."""
     import block_causal_streaming_b200 as wf
     from block_causal_streaming_b200.layer import PagedPoolFp8
     H, D, off = wl.heads, wl.head_dim, wl.chunk_offsets
@@ -292,25 +294,27 @@ def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
     def append_bf16():
         layer.append_range(k, v, chunks, stream)
 
+    def quant_range():
+        wf.kv_append_fp8_chunks(*fp.tensors, 0, 0, wl.num_chunks, k, v, layer.page_tables,
+                                layer.desc, stream)
+
+    def dequant_range():
+        wf.kv_dequant_chunks(*fp.tensors, layer.pool.k, layer.pool.v, 0, 0, wl.num_chunks,
+                             layer.page_tables, layer.desc, stream)
+
+    legs = (quant, dequant, append_bf16, quant_range, dequant_range)
     for _ in range(warmup):
-        quant()
-        dequant()
-        append_bf16()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        for leg in legs:
+            leg()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(legs))]
+           for _ in range(steps)]
     torch.cuda.synchronize(dev)
     for e in evs:
-        torch.sum(flush, dim=(0,), out=sink)
-        e[0].record(stream)
-        quant()
-        e[1].record(stream)
-        torch.sum(flush, dim=(0,), out=sink)
-        e[2].record(stream)
-        dequant()
-        e[3].record(stream)
-        torch.sum(flush, dim=(0,), out=sink)
-        e[4].record(stream)
-        append_bf16()
-        e[5].record(stream)
+        for i, leg in enumerate(legs):
+            torch.sum(flush, dim=(0,), out=sink)
+            e[2 * i].record(stream)
+            leg()
+            e[2 * i + 1].record(stream)
     torch.cuda.synchronize(dev)
     rc = wf.check_status()
     if rc != wf.WF_OK:
@@ -323,13 +327,16 @@ def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
            "bytes_ratio": round(fp8_bytes / bf16_bytes, 4), "peak_gbs": hbm_peak}
     # the plain bf16 append of the same chunks, timed the same way: what one launch per chunk
     # of this size reaches for a pure copy
-    for name, (a, b), nbytes in (("append_fp8", (0, 1), bf16_bytes + fp8_bytes),
-                                 ("dequant", (2, 3), bf16_bytes + fp8_bytes),
-                                 ("append_bf16_reference", (4, 5), 2 * bf16_bytes)):
+    for name, (a, b), nbytes, launches in (
+            ("append_fp8", (0, 1), bf16_bytes + fp8_bytes, wl.num_chunks),
+            ("dequant", (2, 3), bf16_bytes + fp8_bytes, wl.num_chunks),
+            ("append_bf16_reference", (4, 5), 2 * bf16_bytes, wl.num_chunks),
+            ("append_fp8_one_launch", (6, 7), bf16_bytes + fp8_bytes, 1),
+            ("dequant_one_launch", (8, 9), bf16_bytes + fp8_bytes, 1)):
         ms = statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
         gbs = nbytes / (ms / 1e3) / 1e9
         out[name] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4),
-                     "launches": wl.num_chunks}
+                     "launches": launches}
     return out
 
 

@@ -10,7 +10,8 @@ The product is the C-ABI library ``libwf_b200.so`` (declared in ``include/wf.h``
   K/V into other GPUs' pools with a generation flag, and attention that waits for the flags
   (:mod:`.wave` maps the peers' pools between processes);
 * ``wf_kv_append_fp8`` / ``wf_kv_dequant`` -- a chunk's K/V as e4m3 codes with per-(token, head)
-  scales (half the bytes to move), and their conversion back into the bf16 pool;
+  scales (half the bytes to move), and their conversion back into the bf16 pool (``_chunks``:
+  a run of consecutive chunks in one launch);
   ``wf_kv_append_publish_fp8`` / ``wf_kv_dequant_published`` publish those codes into other GPUs'
   FP8 pools with a generation flag, and convert a published chunk once its flag is up;
 * ``wf_qk_quantize_i8`` / ``wf_attn_forward_i8`` -- the INT8 tier: smoothed int8 K and int8 Q
@@ -29,6 +30,7 @@ _ABI_NAMES = (
     "selftest_timeout", "attn_forward_split", "attn_workspace_size",
     "attn_forward_split_noalloc", "kv_append_publish", "attn_forward_published", "ipc_export",
     "ipc_import", "ipc_close", "PoolDst", "kv_append_fp8", "kv_dequant", "KvPoolFp8",
+    "kv_append_fp8_chunks", "kv_dequant_chunks",
     "kv_append_publish_fp8", "kv_dequant_published", "Fp8Dst", "qk_i8_sizes", "qk_quantize_i8",
     "attn_forward_i8", "QkI8", "Segments", "attn_forward_segments",
     "attn_segments_workspace_size",

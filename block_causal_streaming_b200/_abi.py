@@ -29,7 +29,7 @@ EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror",
             "wf_selftest_timeout", "wf_attn_forward_split", "wf_attn_workspace_size",
             "wf_attn_forward_split_noalloc", "wf_kv_append_publish", "wf_attn_forward_published",
             "wf_ipc_export", "wf_ipc_import", "wf_ipc_close", "wf_kv_append_fp8",
-            "wf_kv_dequant", "wf_kv_append_publish_fp8", "wf_kv_dequant_published",
+            "wf_kv_dequant", "wf_kv_append_fp8_chunks", "wf_kv_dequant_chunks", "wf_kv_append_publish_fp8", "wf_kv_dequant_published",
             "wf_qk_i8_sizes", "wf_qk_quantize_i8", "wf_attn_forward_i8",
             "wf_attn_forward_segments", "wf_attn_segments_workspace_size",
             "wf_window_slots", "wf_window_round", "wf_window_round_ring")
@@ -161,6 +161,14 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wf_kv_dequant.argtypes = [ctypes.POINTER(KvPoolFp8), ctypes.POINTER(KvPool), i32, i32,
                                   ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(Wavefront), vp]
     lib.wf_kv_dequant.restype = i32
+    lib.wf_kv_append_fp8_chunks.argtypes = [ctypes.POINTER(KvPoolFp8), i32, i32, i32, vp, vp,
+                                            ctypes.POINTER(ctypes.c_int32),
+                                            ctypes.POINTER(Wavefront), vp]
+    lib.wf_kv_append_fp8_chunks.restype = i32
+    lib.wf_kv_dequant_chunks.argtypes = [ctypes.POINTER(KvPoolFp8), ctypes.POINTER(KvPool), i32,
+                                         i32, i32, ctypes.POINTER(ctypes.c_int32),
+                                         ctypes.POINTER(Wavefront), vp]
+    lib.wf_kv_dequant_chunks.restype = i32
     lib.wf_kv_append_publish_fp8.argtypes = [ctypes.POINTER(KvPoolFp8), vp,
                                              ctypes.POINTER(Fp8Dst), i32, i32, i32, vp, vp,
                                              ctypes.POINTER(ctypes.c_int32),
@@ -457,6 +465,53 @@ def kv_dequant(k_codes, v_codes, k_scale, v_scale, k_pool, v_pool, layer: int, c
                            ctypes.byref(wf.c), _stream_handle(stream))
     if rc != WF_OK:
         raise WfError(rc, "wf_kv_dequant")
+
+
+def kv_append_fp8_chunks(k_codes, v_codes, k_scale, v_scale, layer: int, chunk_begin: int,
+                         chunk_end: int, k, v, page_table, wf: WavefrontDesc, stream=None) -> None:
+    """wf_kv_append_fp8_chunks: kv_append_fp8 of chunks [chunk_begin, chunk_end) in one launch;
+    ``k``, ``v``: those chunks' rows in order, [L, H, D] bf16."""
+    _, _, H, D = _fp8_pool_shape(k_codes, v_codes, k_scale, v_scale)
+    off = wf.chunk_offsets
+    if 0 <= int(chunk_begin) < int(chunk_end) <= len(off) - 1:
+        want = (off[chunk_end] - off[chunk_begin], H, D)
+        for t, n in ((k, "k"), (v, "v")):
+            if tuple(t.shape) != want and not (want[0] == 0 and t.numel() == 0):
+                raise ValueError(f"{n}: chunks [{chunk_begin}, {chunk_end}) need "
+                                 f"[{want[0]}, {H}, {D}], got {tuple(t.shape)}")
+    _check_page_table(page_table, layer, wf)
+    for t, n, d in ((k, "k", "bf16"), (v, "v", "bf16"), (page_table, "page_table", "i32")):
+        _check_tensor(t, n, d)
+    pool = _fp8_pool_struct(k_codes, v_codes, k_scale, v_scale)
+    rc = lib.wf_kv_append_fp8_chunks(ctypes.byref(pool), int(layer), int(chunk_begin),
+                                     int(chunk_end), k.data_ptr(), v.data_ptr(),
+                                     ctypes.cast(ctypes.c_void_p(page_table.data_ptr()),
+                                                 ctypes.POINTER(ctypes.c_int32)),
+                                     ctypes.byref(wf.c), _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_kv_append_fp8_chunks")
+
+
+def kv_dequant_chunks(k_codes, v_codes, k_scale, v_scale, k_pool, v_pool, layer: int,
+                      chunk_begin: int, chunk_end: int, page_table, wf: WavefrontDesc,
+                      stream=None) -> None:
+    """wf_kv_dequant_chunks: kv_dequant of chunks [chunk_begin, chunk_end) in one launch."""
+    geo = _fp8_pool_shape(k_codes, v_codes, k_scale, v_scale)
+    if _pool_shape(k_pool, v_pool) != geo:
+        raise ValueError(f"bf16 pool {tuple(k_pool.shape)} differs from the FP8 pool {geo}")
+    _check_page_table(page_table, layer, wf)
+    for t, n, d in ((k_pool, "k_pool", "bf16"), (v_pool, "v_pool", "bf16"),
+                    (page_table, "page_table", "i32")):
+        _check_tensor(t, n, d)
+    src = _fp8_pool_struct(k_codes, v_codes, k_scale, v_scale)
+    dst = _pool_struct(k_pool, v_pool)
+    rc = lib.wf_kv_dequant_chunks(ctypes.byref(src), ctypes.byref(dst), int(layer),
+                                  int(chunk_begin), int(chunk_end),
+                                  ctypes.cast(ctypes.c_void_p(page_table.data_ptr()),
+                                              ctypes.POINTER(ctypes.c_int32)),
+                                  ctypes.byref(wf.c), _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_kv_dequant_chunks")
 
 
 def kv_append_publish_fp8(k_codes, v_codes, k_scale, v_scale, flags, peers, layer: int,

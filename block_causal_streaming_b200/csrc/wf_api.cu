@@ -791,7 +791,8 @@ int validate_pool_fp8(const wf_kv_pool_fp8_t* pool) {
 // Checks shared by the FP8 calls; on success *t0 / *rows are the chunk's token range and *row its
 // page-table row.
 int fp8_chunk_args(const wf_kv_pool_fp8_t* pool, int layer, int chunk, const int32_t* page_table,
-                   const wf_wavefront_t* wf, int* t0, int* rows, const int32_t** row) {
+                   const wf_wavefront_t* wf, int* t0, int* rows, const int32_t** row,
+                   int chunk_end = -1) {
   int rc = validate_pool_fp8(pool);
   if (rc) return rc;
   wf_kv_pool_t g{pool->k_codes, pool->v_codes, pool->num_pages, pool->page_size, pool->num_heads,
@@ -799,10 +800,12 @@ int fp8_chunk_args(const wf_kv_pool_fp8_t* pool, int layer, int chunk, const int
   int t_kv = 0;
   rc = validate_wavefront(wf, &g, &t_kv);
   if (rc) return rc;
-  if (layer < 0 || chunk < 0 || chunk >= wf->num_chunks || page_table == nullptr)
+  // chunks [chunk, end)
+  const int end = chunk_end < 0 ? chunk + 1 : chunk_end;
+  if (layer < 0 || chunk < 0 || end <= chunk || end > wf->num_chunks || page_table == nullptr)
     return WF_ERR_INVALID_ARG;
   *t0 = wf->chunk_offsets[chunk];
-  *rows = wf->chunk_offsets[chunk + 1] - *t0;
+  *rows = wf->chunk_offsets[end] - *t0;
   *row = page_table + static_cast<int64_t>(layer) * wf->max_pages_per_seq;
   // the quantizer indexes its threads over the (token, head) rows of both tensors with 32-bit
   // integers
@@ -967,6 +970,38 @@ int wf_kv_append_publish_fp8(const wf_kv_pool_fp8_t* pool, uint32_t* flags,
     fp.dst[1 + i].flag = peers[i].flags != nullptr ? peers[i].flags + flag_at : nullptr;
   wfk::wf_publish_flags_kernel<<<1, 32, 0, s>>>(fp);
   return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_kv_append_fp8_chunks(const wf_kv_pool_fp8_t* pool, int layer, int chunk_begin,
+                            int chunk_end, const void* k, const void* v,
+                            const int32_t* page_table, const wf_wavefront_t* wf,
+                            wf_stream_t stream) {
+  int t0 = 0, rows = 0;
+  const int32_t* row = nullptr;
+  if (chunk_end <= chunk_begin) return WF_ERR_INVALID_ARG;
+  const int rc = fp8_chunk_args(pool, layer, chunk_begin, page_table, wf, &t0, &rows, &row,
+                                chunk_end);
+  if (rc) return rc;
+  if (rows == 0) return WF_OK;
+  if (k == nullptr || v == nullptr || !aligned16(k) || !aligned16(v)) return WF_ERR_INVALID_ARG;
+  return launch_quant(pool, nullptr, 0, t0, rows, row, k, v,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int wf_kv_dequant_chunks(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int layer,
+                         int chunk_begin, int chunk_end, const int32_t* page_table,
+                         const wf_wavefront_t* wf, wf_stream_t stream) {
+  int t0 = 0, rows = 0;
+  const int32_t* row = nullptr;
+  if (chunk_end <= chunk_begin) return WF_ERR_INVALID_ARG;
+  int rc = fp8_chunk_args(src, layer, chunk_begin, page_table, wf, &t0, &rows, &row, chunk_end);
+  if (rc) return rc;
+  rc = validate_pool(dst);
+  if (rc) return rc;
+  if (!same_geometry(src, dst)) return WF_ERR_SHAPE;
+  if (rows == 0) return WF_OK;
+  return launch_dequant(src, dst, t0, rows, row, nullptr, 0,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 int wf_kv_dequant(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int layer, int chunk,

@@ -33,7 +33,8 @@
  *     (a page index outside the pool, a bounded wait that ran out) are recorded in a per-device
  *     status word read by wf_check_status.
  *   - Attention computes in bf16 with fp32 accumulation; FP8 appears only in the K/V transport
- *     calls (wf_kv_append_fp8, wf_kv_dequant).  Batch 1, one layer per call.
+ *     calls (wf_kv_append_fp8, wf_kv_dequant and their chunk-range forms).  Batch 1, one layer
+ *     per call.
  */
 #ifndef WF_H_
 #define WF_H_
@@ -308,6 +309,22 @@ int wf_kv_append_fp8(const wf_kv_pool_fp8_t* pool, int layer, int chunk, const v
  */
 int wf_kv_dequant(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int layer, int chunk,
                   const int32_t* page_table, const wf_wavefront_t* wf, wf_stream_t stream);
+
+/*
+ * wf_kv_append_fp8_chunks / wf_kv_dequant_chunks -- wf_kv_append_fp8 / wf_kv_dequant of the
+ * consecutive chunks [chunk_begin, chunk_end) in one launch: the same per-row quantization and
+ * conversion, for chunks written or read together (a round's context, a whole layer).
+ * k, v: the rows of those chunks in order, device bf16 [L][H][D] with L the sum of their
+ * lengths.  Errors as the one-chunk calls; WF_ERR_INVALID_ARG if the range is empty, reversed
+ * or outside the wavefront.
+ */
+int wf_kv_append_fp8_chunks(const wf_kv_pool_fp8_t* pool, int layer, int chunk_begin,
+                            int chunk_end, const void* k, const void* v,
+                            const int32_t* page_table, const wf_wavefront_t* wf,
+                            wf_stream_t stream);
+int wf_kv_dequant_chunks(const wf_kv_pool_fp8_t* src, const wf_kv_pool_t* dst, int layer,
+                         int chunk_begin, int chunk_end, const int32_t* page_table,
+                         const wf_wavefront_t* wf, wf_stream_t stream);
 
 /*
  * FP8 publication (project page, "03 End-to-end KV transport", items 01 "Precision" and 03

@@ -247,3 +247,58 @@ def test_an_fp8_chunk_with_a_page_outside_the_pool_is_not_published():
     assert check_status() == WF_OK
     for f in P.flags:
         assert int(f[LAYER, c]) == 0
+
+
+@pytest.mark.parametrize("wl", CASES[:2], ids=lambda w: w.name)
+def test_chunk_range_forms_equal_the_oracle_and_touch_only_their_rows(wl):
+    """wf_kv_append_fp8_chunks over chunks [1, num_chunks) in one launch: codes and scales of those
+    chunks bit-exact, chunk 0's rows keep the sentinel; wf_kv_dequant_chunks of the same range
+    then writes exactly the oracle's bf16 rows of those chunks and leaves chunk 0's rows alone."""
+    from block_causal_streaming_b200 import kv_append_fp8_chunks, kv_dequant_chunks
+    inp = _with_special_rows(make_inputs(wl))
+    layer, _, k, v = place(wl, inp, append=False, fill=float("nan"))
+    fp = _fp8_pool(wl)
+    off, c0, c1 = wl.chunk_offsets, 1, wl.num_chunks
+    kv_append_fp8_chunks(*fp.tensors, 0, c0, c1, k[off[c0]:off[c1]], v[off[c0]:off[c1]],
+                         layer.page_tables, layer.desc)
+    assert check_status() == WF_OK
+    want = _expected(wl, inp)
+    pt = inp.page_table.numpy()
+    H, D, ps = wl.heads, wl.head_dim, wl.page_size
+    for name, codes, scale in (("k", fp.k_codes, fp.k_scale), ("v", fp.v_codes, fp.v_scale)):
+        _, _, q_codes, q_scale = want[name]
+        w_codes = np.full((wl.num_pages, ps, H, D), SENTINEL_CODE, np.uint8)
+        w_scale = np.full((wl.num_pages, ps, H), np.nan, np.float32)
+        oracle.scatter_chunk(w_codes, pt, off[c0], q_codes[off[c0]:off[c1]])
+        oracle.scatter_chunk(w_scale, pt, off[c0], q_scale[off[c0]:off[c1]])
+        assert np.array_equal(codes.cpu().numpy(), w_codes), f"{name} codes"
+        assert np.array_equal(scale.cpu().numpy().view(np.int32), w_scale.view(np.int32)), \
+            f"{name} scales"
+    kv_dequant_chunks(*fp.tensors, layer.pool.k, layer.pool.v, 0, c0, c1, layer.page_tables,
+                      layer.desc)
+    assert check_status() == WF_OK
+    for name, pool in (("k", layer.pool.k), ("v", layer.pool.v)):
+        _, _, q_codes, q_scale = want[name]
+        deq = ofp8.dequantize_rows(q_codes, q_scale).view(torch.int16).numpy()
+        got = oracle.gather_logical(pool.cpu().view(torch.int16).numpy(), pt, wl.t_kv)
+        assert np.array_equal(got[off[c0]:off[c1]], deq[off[c0]:off[c1]]), f"{name} dequantized"
+        assert np.all(got[:off[c0]] == np.int16(0x7FC0)), f"{name}: chunk 0 rows were written"
+
+
+def test_chunk_range_forms_reject_empty_and_reversed_ranges():
+    from block_causal_streaming_b200 import (WF_ERR_INVALID_ARG, WfError, kv_append_fp8_chunks,
+                                             kv_dequant_chunks)
+    wl = CASES[0]
+    inp = make_inputs(wl)
+    layer, _, k, v = place(wl, inp, append=False)
+    fp = _fp8_pool(wl)
+    for c0, c1 in ((1, 1), (2, 1), (0, wl.num_chunks + 1)):
+        with pytest.raises(WfError) as e:
+            kv_append_fp8_chunks(*fp.tensors, 0, c0, c1, k[:0], v[:0], layer.page_tables,
+                                 layer.desc)
+        assert e.value.code == WF_ERR_INVALID_ARG
+        with pytest.raises(WfError) as e:
+            kv_dequant_chunks(*fp.tensors, layer.pool.k, layer.pool.v, 0, c0, c1,
+                              layer.page_tables, layer.desc)
+        assert e.value.code == WF_ERR_INVALID_ARG
+    assert check_status() == WF_OK
