@@ -30,7 +30,7 @@ _ABI_NAMES = (
     "selftest_timeout", "attn_forward_split", "attn_workspace_size",
     "attn_forward_split_noalloc", "kv_append_publish", "attn_forward_published", "ipc_export",
     "ipc_import", "ipc_close", "PoolDst", "kv_append_fp8", "kv_dequant", "KvPoolFp8",
-    "kv_append_fp8_chunks", "kv_dequant_chunks",
+    "kv_append_fp8_chunks", "kv_dequant_chunks", "attn_split_plan",
     "kv_append_publish_fp8", "kv_dequant_published", "Fp8Dst", "qk_i8_sizes", "qk_quantize_i8",
     "attn_forward_i8", "QkI8", "Segments", "attn_forward_segments",
     "attn_segments_workspace_size",

@@ -29,7 +29,8 @@ EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror",
             "wf_selftest_timeout", "wf_attn_forward_split", "wf_attn_workspace_size",
             "wf_attn_forward_split_noalloc", "wf_kv_append_publish", "wf_attn_forward_published",
             "wf_ipc_export", "wf_ipc_import", "wf_ipc_close", "wf_kv_append_fp8",
-            "wf_kv_dequant", "wf_kv_append_fp8_chunks", "wf_kv_dequant_chunks", "wf_kv_append_publish_fp8", "wf_kv_dequant_published",
+            "wf_kv_dequant", "wf_kv_append_fp8_chunks", "wf_kv_dequant_chunks",
+            "wf_attn_split_plan", "wf_kv_append_publish_fp8", "wf_kv_dequant_published",
             "wf_qk_i8_sizes", "wf_qk_quantize_i8", "wf_attn_forward_i8",
             "wf_attn_forward_segments", "wf_attn_segments_workspace_size",
             "wf_window_slots", "wf_window_round", "wf_window_round_ring")
@@ -155,6 +156,10 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wf_ipc_close.restype = i32
     lib.wf_attn_workspace_size.argtypes = [ctypes.POINTER(Wavefront), i32, i32, i32]
     lib.wf_attn_workspace_size.restype = ctypes.c_size_t
+    lib.wf_attn_split_plan.argtypes = [ctypes.POINTER(Wavefront), i32, i32, i32,
+                                       ctypes.POINTER(ctypes.c_int32),
+                                       ctypes.POINTER(ctypes.c_int32)]
+    lib.wf_attn_split_plan.restype = i32
     lib.wf_kv_append_fp8.argtypes = [ctypes.POINTER(KvPoolFp8), i32, i32, vp, vp,
                                      ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(Wavefront), vp]
     lib.wf_kv_append_fp8.restype = i32
@@ -671,6 +676,17 @@ def attn_workspace_size(wf: WavefrontDesc, num_heads: int, head_dim: int, splits
     """wf_attn_workspace_size: bytes of workspace attn_forward_split needs (0: none)."""
     return int(lib.wf_attn_workspace_size(ctypes.byref(wf.c), int(num_heads), int(head_dim),
                                           int(splits)))
+
+
+def attn_split_plan(wf: WavefrontDesc, num_heads: int, splits: int = 0, num_sms: int = 0):
+    """wf_attn_split_plan: (parts, tail_units) -- every unit in ``parts`` parts, the last
+    ``tail_units`` units of the dispatch order in parts + 1.  ``num_sms`` 0: the current device."""
+    parts, tail = ctypes.c_int32(0), ctypes.c_int32(0)
+    rc = lib.wf_attn_split_plan(ctypes.byref(wf.c), int(num_heads), int(splits), int(num_sms),
+                                ctypes.byref(parts), ctypes.byref(tail))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_attn_split_plan")
+    return parts.value, tail.value
 
 
 def attn_forward_split(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: float, out,

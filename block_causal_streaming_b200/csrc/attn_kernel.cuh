@@ -102,11 +102,13 @@ struct AttnParams {
   int nqc;                          // non-empty query chunks
   int qc_row_end[kMaxQChunks];      // exclusive end row of query chunk i (query-row space)
   int qc_kv_end[kMaxQChunks];       // number of visible keys for rows of query chunk i
-  // Key splits: with n_splits > 1 every unit runs as n_splits CTAs over consecutive parts of its
-  // key tiles, and each writes its normalised partial output and log-sum-exp instead of `out`.
+  // Key splits: every unit runs as n_splits CTAs over consecutive parts of its key tiles -- the
+  // last n_tail units (in dispatch order) as n_splits + 1 -- and a unit with more than one part
+  // writes, per part, its normalised partial output and log-sum-exp instead of `out`.
   int n_splits;
-  float* part_o;                    // fp32 [n_splits][T_q][H][D]
-  float* part_lse;                  // fp32 [n_splits][H][T_q], natural log; -inf: no key seen
+  int n_tail;
+  float* part_o;                    // fp32 [parts][T_q][H][D], parts = n_splits (+1 with a tail)
+  float* part_lse;                  // fp32 [parts][H][T_q], natural log; -inf: no key seen
   // Published chunks (one-way K/V publication between GPUs): with flags != null the keys of
   // chunk c are loaded only after flags[c] has reached flag_gen.  chunk_end[c]: exclusive end
   // token of chunk c in the logical key order.
@@ -198,8 +200,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto bar = [&](int i) -> uint32_t { return base + L::BAR_OFF + 8u * static_cast<uint32_t>(i); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int unit = blockIdx.x / p.n_splits;
-  const int split = blockIdx.x - unit * p.n_splits;
+  // unit, part and parts of this CTA: (U - n_tail) units of n_splits parts, then n_tail units
+  // of n_splits + 1
+  const int n_plain = p.n_pairs * p.H - p.n_tail;
+  const int b_id = static_cast<int>(blockIdx.x);
+  int unit, split, n_parts;
+  if (b_id < n_plain * p.n_splits) {
+    n_parts = p.n_splits;
+    unit = b_id / n_parts;
+    split = b_id - unit * n_parts;
+  } else {
+    n_parts = p.n_splits + 1;
+    const int t = b_id - n_plain * p.n_splits;
+    unit = n_plain + t / n_parts;
+    split = t - (unit - n_plain) * n_parts;
+  }
   // Heads are dispatched in groups of head_group: every row block of one group, longest first,
   // heads fastest, before the next group -- so many CTAs read one head's keys at about the same
   // time, whatever H is.
@@ -211,10 +226,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int last_row = min(m0 + kNQT * kBM, p.T_q) - 1;
   const int n_max = kv_end_of_row(p, last_row);        // keys any row of this unit may see
   const int n_tiles = (n_max + BN - 1) / BN;           // key tiles of the unit
-  // This CTA's part of them: tiles [kb, kb + nk).  The host keeps n_splits <= n_tiles of every
+  // This CTA's part of them: tiles [kb, kb + nk).  The host keeps n_parts <= n_tiles of every
   // unit, so nk >= 1.  Tile j below is local; its keys start at (kb + j) * BN.
-  const int kb = static_cast<int>(static_cast<int64_t>(split) * n_tiles / p.n_splits);
-  const int nk = static_cast<int>(static_cast<int64_t>(split + 1) * n_tiles / p.n_splits) - kb;
+  const int kb = static_cast<int>(static_cast<int64_t>(split) * n_tiles / n_parts);
+  const int nk = static_cast<int>(static_cast<int64_t>(split + 1) * n_tiles / n_parts) - kb;
 
   const WaitCtx w{cta_abort, p.grid_abort, p.status, p.launch_id, 6 /* WF_ERR_TIMEOUT */,
                   kWaitTimeoutNs};
@@ -363,7 +378,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // O / l: bf16 into `out`, or -- for one key split of a unit -- fp32 into the partials,
         // with O = 0 and lse = -inf when no key of the split is visible to the row.
         tc_fence_after();
-        const bool part = p.n_splits > 1;
+        const bool part = n_parts > 1;
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
         const bool live = row_g < p.T_q;
         const size_t orow = static_cast<size_t>(row_g) * p.H + head;

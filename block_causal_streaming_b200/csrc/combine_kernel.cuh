@@ -1,6 +1,7 @@
 // combine_kernel.cuh -- merge of the key splits of a split attention launch (sm_100a).
 //
-// When a unit's key range is split over S CTAs, CTA s writes O_s = (sum over its keys of
+// When a unit's key range is split over S CTAs (S may differ between units: a launch can give its
+// last units one part more), CTA s writes O_s = (sum over its keys of
 // p_j v_j) / l_s and lse_s = log l_s (natural log, max folded in; -inf when none of its keys is
 // visible to the row).  The softmax over all keys is then
 //   lse = log sum_s exp(lse_s),   out = sum_s exp(lse_s - lse) O_s,
@@ -16,11 +17,31 @@ namespace wfk {
 
 constexpr int kCombineThreads = 256;
 
-// One warp per (query row, head); lane i owns head-dim columns [i D/32, (i+1) D/32).
+// Which rows were split, and into how many parts: the unit layout of the attention launch
+// (units of unit_rows query rows x one head, numbered in its dispatch order).
+struct CombinePlan {
+  int n_splits;      // parts of the first units
+  int n_tail;        // the last n_tail units have n_splits + 1 parts
+  int n_pairs;       // row blocks per head
+  int head_group;    // heads per dispatch group
+  int unit_rows;     // query rows per unit
+};
+
+// Parts of the unit that holds (row, head) -- the inverse of the attention kernel's unit order.
+__device__ __forceinline__ int combine_parts(const CombinePlan& c, int row, int head, int H) {
+  const int pair = row / c.unit_rows;
+  const int group = head / c.head_group;
+  const int unit = group * c.n_pairs * c.head_group + (c.n_pairs - 1 - pair) * c.head_group +
+                   head % c.head_group;
+  return unit >= c.n_pairs * H - c.n_tail ? c.n_splits + 1 : c.n_splits;
+}
+
+// One warp per (query row, head); lane i owns head-dim columns [i D/32, (i+1) D/32).  Rows of a
+// unit that ran in one part are final already and are skipped.
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads)
     wf_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                      int n_splits, int T_q, int H, __nv_bfloat16* __restrict__ out,
+                      CombinePlan plan, int T_q, int H, __nv_bfloat16* __restrict__ out,
                       float* __restrict__ lse) {
   constexpr int V = D / 32;   // 4 columns (one float4) at D = 128, 2 at D = 64
   static_assert(V == 2 || V == 4, "head_dim 64 or 128");
@@ -28,6 +49,8 @@ __global__ void __launch_bounds__(kCombineThreads)
   const int lane = threadIdx.x & 31;
   if (item >= static_cast<int64_t>(T_q) * H) return;
   const int row = static_cast<int>(item / H), head = static_cast<int>(item - int64_t(row) * H);
+  const int n_splits = combine_parts(plan, row, head, H);
+  if (n_splits < 2) return;
 
   float mx = -INFINITY;
   for (int s = 0; s < n_splits; ++s)

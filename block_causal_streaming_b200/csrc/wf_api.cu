@@ -10,6 +10,8 @@
 #include <cstring>
 #include <algorithm>
 #include <mutex>
+#include <vector>
+#include <queue>
 
 #include "../../include/wf.h"
 #include "append_kernel.cuh"
@@ -27,9 +29,10 @@ __device__ int g_wf_status = 0;
 __device__ unsigned g_wf_abort = 0;
 
 // Scratch of wf_attn_forward_split_noalloc: one static array per device, so that entry point
-// needs no allocation.  96 MiB holds the partial results of 3 key splits of a 4680-row, 12-head,
-// head_dim-128 call (3 x 4680 x 12 x 129 x 4 B = 86.9 MB); larger plans are rejected.
-constexpr size_t kScratchBytes = size_t(96) << 20;
+// needs no allocation.  128 MiB holds the partial results of the library's plan for a 4680-row,
+// 12-head, head_dim-128 call -- 3 key splits, the last units 4 (4 x 4680 x 12 x 129 x 4 B =
+// 115.9 MB); larger plans are rejected.
+constexpr size_t kScratchBytes = size_t(128) << 20;
 __device__ __align__(256) unsigned char g_wf_scratch[kScratchBytes];
 
 namespace {
@@ -275,31 +278,114 @@ int max_splits(const QueryPlan& qp) {
 
 size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 
-// part_o: fp32 [S][T_q][H][D], then part_lse: fp32 [S][H][T_q].
+// part_o: fp32 [S][T_q][H][D], then part_lse: fp32 [S][H][T_q] (S: the plan's most parts).
 size_t split_workspace_bytes(const QueryPlan& qp, int H, int D, int S) {
   if (S <= 1) return 0;
   const size_t rows = static_cast<size_t>(S) * qp.t_q * H;
   return align256(rows * D * sizeof(float)) + align256(rows * sizeof(float));
 }
 
-// Key splits per unit, from how full the last wave of CTAs is.  With U units on G SMs (one CTA
-// per SM) a single pass fills (U/G) / ceil(U/G) of the SM-time; S splits fill
-// (S U/G) / ceil(S U/G) but pay S - 1 more prologues per unit and a merge pass.  Split only a
-// grid shorter than two waves whose last wave is less than 80 % full, into the fewest splits
-// that fill 90 %.  (Measured on one Wave-Parallelism rank's call, 228 units on 148 SMs:
-// S = 1, 2, 3, 5, 6, 16 -> 1.18, 1.22, 1.16, 1.16, 1.35, 1.53 ms: tail waves cost about what
-// this fill predicts, and further splits only add overhead.)
-int choose_splits(const QueryPlan& qp, int H, int num_sms) {
+// A split plan: every unit runs in S parts (CTAs over consecutive key tiles), the last `tail`
+// units of the dispatch order in S + 1.
+struct SplitPlan {
+  int S = 1;
+  int tail = 0;
+  int parts() const { return tail > 0 ? S + 1 : S; }
+};
+
+// Length in tile-times of one launch under `plan`: CTAs in dispatch order go to the SM that
+// frees first (the hardware's in-order block dispatch), each costing its key tiles plus a
+// prologue/epilogue of kCtaOverhead tiles; a plan with parts adds the merge pass, about
+// kMergePerPart tile-times per million (row, head, part) items.  (Calibrated on one
+// Wave-Parallelism rank's call on a B200: ~3 us of prologue per CTA, ~1.3 us per tile, the
+// merge of 3 x 4680 x 12 parts ~29 us.)
+constexpr double kCtaOverhead = 2.5, kMergePerPart = 130.0;
+double plan_cost(const QueryPlan& qp, int H, int num_sms, const SplitPlan& plan) {
+  const int n_pairs = num_pairs(qp);
+  const int hg = head_group(H);
+  const int units = n_pairs * H;
+  std::vector<double> sm(static_cast<size_t>(num_sms), 0.0);
+  std::priority_queue<std::pair<double, int>, std::vector<std::pair<double, int>>,
+                      std::greater<std::pair<double, int>>> free_at;
+  for (int i = 0; i < num_sms; ++i) free_at.push({0.0, i});
+  double makespan = 0.0, merge_items = 0.0;
+  for (int u = 0; u < units; ++u) {
+    const int in_group = u % (n_pairs * hg);
+    const int pair = n_pairs - 1 - in_group / hg;
+    const int n = unit_tiles(qp, pair);
+    const int parts = u >= units - plan.tail ? plan.S + 1 : plan.S;
+    const int rows = std::min((pair + 1) * kUnitRows, qp.t_q) - pair * kUnitRows;
+    if (parts > 1) merge_items += static_cast<double>(rows) * parts;
+    for (int s = 0; s < parts; ++s) {
+      const int nk = static_cast<int>(static_cast<int64_t>(s + 1) * n / parts) -
+                     static_cast<int>(static_cast<int64_t>(s) * n / parts);
+      auto top = free_at.top();
+      free_at.pop();
+      const double end = top.first + nk + kCtaOverhead;
+      makespan = std::max(makespan, end);
+      free_at.push({end, top.second});
+    }
+  }
+  return makespan + kMergePerPart * merge_items / 1e6;
+}
+
+// Key splits per unit, for grids shorter than two waves (one CTA per SM): of the plans with S
+// parts per unit -- one part, or S >= 2 alone or with the last units given one part more so
+// that the CTAs fill whole waves -- the one plan_cost finds shortest.  The choice is cached per query layout.
+// (Measured on one Wave-Parallelism rank's call, 228 units on 148 SMs, uniform S = 1, 2, 3, 4,
+// 5, 6, 16 -> 1.18, 1.22, 1.16, 1.27, 1.22, 1.32, 1.53 ms with an earlier kernel: tail waves
+// cost about what this model predicts.)
+SplitPlan auto_plan(const QueryPlan& qp, int H, int num_sms) {
   const int64_t units = static_cast<int64_t>(num_pairs(qp)) * H;
-  auto fill = [&](int S) {
-    const double waves = static_cast<double>(units) * S / num_sms;
-    return waves / std::ceil(waves);
+  SplitPlan best;
+  if (units >= 2 * static_cast<int64_t>(num_sms) || units * kMaxSplits > INT32_MAX / 2)
+    return best;
+  struct Entry {
+    QueryPlan qp;
+    int H, sms;
+    SplitPlan plan;
   };
-  if (units >= 2 * static_cast<int64_t>(num_sms) || fill(1) >= 0.8) return 1;
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  auto same = [&](const Entry& e) {
+    if (e.H != H || e.sms != num_sms || e.qp.t_q != qp.t_q || e.qp.nqc != qp.nqc) return false;
+    for (int c = 0; c < qp.nqc; ++c)
+      if (e.qp.row_end[c] != qp.row_end[c] || e.qp.kv_end[c] != qp.kv_end[c]) return false;
+    return true;
+  };
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : cache)
+      if (same(e)) return e.plan;
+  }
   const int cap = max_splits(qp);
-  for (int S = 2; S <= cap; ++S)
-    if (fill(S) >= 0.9) return S;
-  return 1;
+  double best_cost = plan_cost(qp, H, num_sms, best);
+  for (int S = 1; S <= cap; ++S) {
+    const int64_t ctas = units * S;
+    const int64_t fill = (ctas + num_sms - 1) / num_sms * num_sms - ctas;
+    for (const int64_t tail : {int64_t{0}, fill}) {
+      // (a tail on S = 1 would mix whole and split units; every plan keeps all units split or
+      // none)
+      if (S == 1 || tail > units || (tail > 0 && S + 1 > cap)) continue;
+      const SplitPlan cand{S, static_cast<int>(tail)};
+      const double cost = plan_cost(qp, H, num_sms, cand);
+      if (cost < best_cost) {
+        best_cost = cost;
+        best = cand;
+      }
+    }
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= 32) cache.erase(cache.begin());
+  cache.push_back({qp, H, num_sms, best});
+  return best;
+}
+
+// The plan of a call: `splits` > 0 asks for that many parts in every unit (capped so that every
+// part has a key tile); 0 lets the library choose.
+SplitPlan plan_splits(const QueryPlan& qp, int H, int num_sms, int splits) {
+  if (splits > 0) return SplitPlan{std::min(splits, max_splits(qp)), 0};
+  return auto_plan(qp, H, num_sms);
 }
 
 // Device address of g_wf_scratch on the current device, looked up once per device.
@@ -427,10 +513,11 @@ int prepare_common(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* p
   return WF_OK;
 }
 
-// Point the launch at a workspace holding S partial results.
-void set_split_buffers(AttnLaunch* L, int S, void* workspace) {
-  const size_t rows = static_cast<size_t>(S) * L->qp.t_q * L->p.H;
-  L->p.n_splits = S;
+// Point the launch at a workspace holding the plan's partial results.
+void set_split_buffers(AttnLaunch* L, const SplitPlan& plan, void* workspace) {
+  const size_t rows = static_cast<size_t>(plan.parts()) * L->qp.t_q * L->p.H;
+  L->p.n_splits = plan.S;
+  L->p.n_tail = plan.tail;
   L->p.part_o = static_cast<float*>(workspace);
   L->p.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                            align256(rows * L->D * sizeof(float)));
@@ -440,7 +527,7 @@ int launch_attention(AttnLaunch* L, cudaStream_t s) {
   wfk::AttnParams& p = L->p;
   p.launch_id = g_launch_counter.fetch_add(1);
   if (p.launch_id == 0) p.launch_id = g_launch_counter.fetch_add(1);
-  const int64_t grid = static_cast<int64_t>(p.n_pairs) * p.H * p.n_splits;
+  const int64_t grid = static_cast<int64_t>(p.n_pairs) * p.H * p.n_splits + p.n_tail;
   const unsigned g = static_cast<unsigned>(grid);
   const bool wait = p.flags != nullptr;
   if (L->D == 128 && !wait)
@@ -453,16 +540,17 @@ int launch_attention(AttnLaunch* L, cudaStream_t s) {
   else
     wfk::wf_attn_fwd_kernel<64, true><<<g, wfk::kAttnThreads, wfk::AttnSmem<64>::ALLOC, s>>>(p);
   if (cudaGetLastError() != cudaSuccess) return WF_ERR_CUDA;
-  if (p.n_splits > 1) {
+  if (p.n_splits > 1 || p.n_tail > 0) {
     const int64_t threads = static_cast<int64_t>(p.T_q) * p.H * 32;
     const unsigned blocks =
         static_cast<unsigned>((threads + wfk::kCombineThreads - 1) / wfk::kCombineThreads);
+    const wfk::CombinePlan cp{p.n_splits, p.n_tail, p.n_pairs, p.head_group, kUnitRows};
     if (L->D == 128)
       wfk::wf_combine_kernel<128><<<blocks, wfk::kCombineThreads, 0, s>>>(
-          p.part_o, p.part_lse, p.n_splits, p.T_q, p.H, p.out, L->lse_out);
+          p.part_o, p.part_lse, cp, p.T_q, p.H, p.out, L->lse_out);
     else
       wfk::wf_combine_kernel<64><<<blocks, wfk::kCombineThreads, 0, s>>>(
-          p.part_o, p.part_lse, p.n_splits, p.T_q, p.H, p.out, L->lse_out);
+          p.part_o, p.part_lse, cp, p.T_q, p.H, p.out, L->lse_out);
     if (cudaGetLastError() != cudaSuccess) return WF_ERR_CUDA;
   }
   return WF_OK;
@@ -549,14 +637,33 @@ size_t wf_attn_workspace_size(const wf_wavefront_t* wf, int num_heads, int head_
   if (wf == nullptr || num_heads < 1 || (head_dim != 64 && head_dim != 128) || splits < 0 ||
       query_plan(wf, &qp) != WF_OK || qp.t_q == 0)
     return 0;
-  int S = splits;
-  if (S == 0) {
+  int sms = 0;
+  if (splits == 0) {
     DeviceState* d = nullptr;
     if (device_state(&d) != WF_OK) return 0;
-    S = choose_splits(qp, num_heads, d->num_sms);
+    sms = d->num_sms;
   }
-  S = std::min(S, max_splits(qp));
-  return split_workspace_bytes(qp, num_heads, head_dim, S);
+  const SplitPlan plan = plan_splits(qp, num_heads, sms, splits);
+  return split_workspace_bytes(qp, num_heads, head_dim, plan.parts());
+}
+
+int wf_attn_split_plan(const wf_wavefront_t* wf, int num_heads, int splits, int num_sms,
+                       int32_t* parts, int32_t* tail_units) {
+  if (wf == nullptr || parts == nullptr || tail_units == nullptr || splits < 0 || num_heads < 1 ||
+      num_sms < 0)
+    return WF_ERR_INVALID_ARG;
+  QueryPlan qp;
+  if (query_plan(wf, &qp) != WF_OK || qp.t_q == 0) return WF_ERR_SHAPE;
+  if (splits == 0 && num_sms == 0) {
+    DeviceState* d = nullptr;
+    const int rc = device_state(&d);
+    if (rc) return rc;
+    num_sms = d->num_sms;
+  }
+  const SplitPlan plan = plan_splits(qp, num_heads, num_sms, splits);
+  *parts = plan.S;
+  *tail_units = plan.tail;
+  return WF_OK;
 }
 
 int wf_attn_forward_split(const void* q, const wf_kv_pool_t* kv_pages,
@@ -567,13 +674,12 @@ int wf_attn_forward_split(const void* q, const wf_kv_pool_t* kv_pages,
   AttnLaunch L;
   const int rc = prepare_attention(q, kv_pages, page_table_row, wf, scale, out, lse_or_null, &L);
   if (rc || L.p.T_q == 0) return rc;
-  int S = splits > 0 ? splits : choose_splits(L.qp, L.p.H, L.d->num_sms);
-  S = std::min(S, max_splits(L.qp));
-  if (S > 1) {
-    const size_t need = split_workspace_bytes(L.qp, L.p.H, L.D, S);
+  const SplitPlan plan = plan_splits(L.qp, L.p.H, L.d->num_sms, splits);
+  if (plan.parts() > 1) {
+    const size_t need = split_workspace_bytes(L.qp, L.p.H, L.D, plan.parts());
     if (workspace == nullptr || !aligned16(workspace)) return WF_ERR_INVALID_ARG;
     if (workspace_bytes < need) return WF_ERR_CAPACITY;
-    set_split_buffers(&L, S, workspace);
+    set_split_buffers(&L, plan, workspace);
   }
   return launch_attention(&L, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -590,13 +696,12 @@ int wf_attn_forward_segments(const void* q, const wf_kv_pool_t* kv_pages,
   if (rc) return rc;
   rc = prepare_common(q, kv_pages, page_table_row, scale, out, lse_or_null, &L);
   if (rc || L.p.T_q == 0) return rc;
-  int S = splits > 0 ? splits : choose_splits(L.qp, L.p.H, L.d->num_sms);
-  S = std::min(S, max_splits(L.qp));
-  if (S > 1) {
-    const size_t need = split_workspace_bytes(L.qp, L.p.H, L.D, S);
+  const SplitPlan plan = plan_splits(L.qp, L.p.H, L.d->num_sms, splits);
+  if (plan.parts() > 1) {
+    const size_t need = split_workspace_bytes(L.qp, L.p.H, L.D, plan.parts());
     if (workspace == nullptr || !aligned16(workspace)) return WF_ERR_INVALID_ARG;
     if (workspace_bytes < need) return WF_ERR_CAPACITY;
-    set_split_buffers(&L, S, workspace);
+    set_split_buffers(&L, plan, workspace);
   }
   return launch_attention(&L, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -613,14 +718,14 @@ size_t wf_attn_segments_workspace_size(const wf_segments_t* segments, int num_he
   wf_segments_t s = *segments;
   s.max_pages_per_seq = INT32_MAX;          // capacity is checked by the attention call
   if (segments_plan(&s, &geo, &qp) != WF_OK || qp.t_q == 0) return 0;
-  int S = splits;
-  if (S == 0) {
+  int sms = 0;
+  if (splits == 0) {
     DeviceState* d = nullptr;
     if (device_state(&d) != WF_OK) return 0;
-    S = choose_splits(qp, num_heads, d->num_sms);
+    sms = d->num_sms;
   }
-  S = std::min(S, max_splits(qp));
-  return split_workspace_bytes(qp, num_heads, head_dim, S);
+  const SplitPlan plan = plan_splits(qp, num_heads, sms, splits);
+  return split_workspace_bytes(qp, num_heads, head_dim, plan.parts());
 }
 
 int wf_attn_forward_split_noalloc(const void* q, const wf_kv_pool_t* kv_pages,
@@ -631,14 +736,14 @@ int wf_attn_forward_split_noalloc(const void* q, const wf_kv_pool_t* kv_pages,
   AttnLaunch L;
   int rc = prepare_attention(q, kv_pages, page_table_row, wf, scale, out, lse_or_null, &L);
   if (rc || L.p.T_q == 0) return rc;
-  int S = splits > 0 ? splits : choose_splits(L.qp, L.p.H, L.d->num_sms);
-  S = std::min(S, max_splits(L.qp));
-  if (S > 1) {
-    if (split_workspace_bytes(L.qp, L.p.H, L.D, S) > kScratchBytes) return WF_ERR_CAPACITY;
+  const SplitPlan plan = plan_splits(L.qp, L.p.H, L.d->num_sms, splits);
+  if (plan.parts() > 1) {
+    if (split_workspace_bytes(L.qp, L.p.H, L.D, plan.parts()) > kScratchBytes)
+      return WF_ERR_CAPACITY;
     void* scratch = nullptr;
     rc = scratch_address(&scratch);
     if (rc) return rc;
-    set_split_buffers(&L, S, scratch);
+    set_split_buffers(&L, plan, scratch);
   }
   return launch_attention(&L, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -709,13 +814,12 @@ int wf_attn_forward_published(const void* q, const wf_kv_pool_t* kv_pages,
   AttnLaunch L;
   const int rc = prepare_attention(q, kv_pages, page_table_row, wf, scale, out, lse_or_null, &L);
   if (rc || L.p.T_q == 0) return rc;
-  int S = splits > 0 ? splits : choose_splits(L.qp, L.p.H, L.d->num_sms);
-  S = std::min(S, max_splits(L.qp));
-  if (S > 1) {
-    const size_t need = split_workspace_bytes(L.qp, L.p.H, L.D, S);
+  const SplitPlan plan = plan_splits(L.qp, L.p.H, L.d->num_sms, splits);
+  if (plan.parts() > 1) {
+    const size_t need = split_workspace_bytes(L.qp, L.p.H, L.D, plan.parts());
     if (workspace == nullptr || !aligned16(workspace)) return WF_ERR_INVALID_ARG;
     if (workspace_bytes < need) return WF_ERR_CAPACITY;
-    set_split_buffers(&L, S, workspace);
+    set_split_buffers(&L, plan, workspace);
   }
   L.p.flags = flags_row;
   L.p.flag_gen = generation;

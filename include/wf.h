@@ -141,7 +141,9 @@ int wf_attn_forward(const void* q, const wf_kv_pool_t* kv_pages, const int32_t* 
  * of the unit's key tiles; a second kernel merges them (out = sum_s exp(lse_s - lse) O_s).
  * Arguments and result as wf_attn_forward, plus:
  *   splits           S >= 1 key splits per unit (capped at 16 and at the key tiles of the
- *                    smallest unit), or 0 to let the library pick S from a model of the grid.
+ *                    smallest unit), or 0 to let the library plan them from a model of the
+ *                    grid (wf_attn_split_plan): S parts per unit, the last units of the
+ *                    dispatch order possibly S + 1, so that the CTAs fill whole waves.
  *   workspace        device memory, 16-byte aligned, caller-owned, at least
  *                    wf_attn_workspace_size(wf, H, D, splits) bytes; may be null when that
  *                    size is 0 (S = 1 runs exactly wf_attn_forward's single pass).
@@ -156,11 +158,12 @@ int wf_attn_forward_split(const void* q, const wf_kv_pool_t* kv_pages,
 
 /*
  * wf_attn_forward_split_noalloc -- wf_attn_forward_split without a caller workspace: the partial
- * results go to a static 96 MiB (100 663 296-byte) array the library keeps in device memory, one
+ * results go to a static 128 MiB (134 217 728-byte) array the library keeps in device memory, one
  * per device, so the call allocates nothing.  No counterpart on the pages: it exists for callers
  * that cannot hand over device memory.  Arguments and result as wf_attn_forward_split without
- * `workspace` / `workspace_bytes`; WF_ERR_CAPACITY when the plan needs more than the 96 MiB
- * (S * T_q * H * (D + 1) * 4 bytes; pass a smaller `splits` or use wf_attn_forward_split).
+ * `workspace` / `workspace_bytes`; WF_ERR_CAPACITY when the plan needs more than the 128 MiB
+ * (P * T_q * H * (D + 1) * 4 bytes, P the plan's most parts; pass a smaller `splits` or use
+ * wf_attn_forward_split).
  * Sharing: every call on a device uses the same array.  Calls that may run at the same time --
  * on different streams of one device, or from several host threads without ordering -- race on
  * it and may return wrong results; order them on one stream (the array is only read by the
@@ -174,10 +177,23 @@ int wf_attn_forward_split_noalloc(const void* q, const wf_kv_pool_t* kv_pages,
 /*
  * wf_attn_workspace_size -- bytes of workspace wf_attn_forward_split needs for this wavefront,
  * head count, head_dim and `splits` (0: the library's choice on the current device):
- * S * T_q * H * (D + 1) * 4 bytes (fp32 partial outputs and log-sum-exps, each rounded up to 256)
- * when S > 1, else 0.  Also 0 for invalid arguments (the forward call then reports the error).
+ * P * T_q * H * (D + 1) * 4 bytes (fp32 partial outputs and log-sum-exps, each rounded up to 256)
+ * with P the plan's largest part count, when some unit is split, else 0.  Also 0 for invalid
+ * arguments (the forward call then reports the error).
  */
 size_t wf_attn_workspace_size(const wf_wavefront_t* wf, int num_heads, int head_dim, int splits);
+
+/*
+ * wf_attn_split_plan -- the split plan wf_attn_forward_split uses for this wavefront and head
+ * count: every unit (256 query rows x one head) in *parts parts, the last *tail_units units of the
+ * dispatch order in *parts + 1.  splits > 0 gives that uniform plan (capped as above); 0 the
+ * library's choice for num_sms SMs (0: the current device's).  Host-only when num_sms > 0.
+ * Errors: WF_ERR_INVALID_ARG for null pointers or splits < 0; WF_ERR_SHAPE for an invalid
+ * wavefront or one without query rows; WF_ERR_NO_DEVICE if num_sms is 0 and no sm_100 device is
+ * current.
+ */
+int wf_attn_split_plan(const wf_wavefront_t* wf, int num_heads, int splits, int num_sms,
+                       int32_t* parts, int32_t* tail_units);
 
 /* ---------------------------------------------------------------------------------------------
  * One-way K/V publication between GPUs (Wave Parallelism).  Every GPU owns one chunk of the

@@ -115,3 +115,25 @@ def test_sixteen_splits_the_maximum():
         assert check_status() == WF_OK
         assert_parity(out.float().cpu().numpy(), ref, f"S={splits}")
         np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=2e-3)
+
+
+def test_library_plan_with_a_tail_of_units_split_once_more_every_element():
+    """A wavefront for which the library's plan (on a 148-SM B200) gives every unit 3 parts and
+    the last units of the dispatch order 4, so that the CTAs fill whole waves: every element and
+    every lse against the oracle, and rows of the units left whole by another plan equal too."""
+    from block_causal_streaming_b200 import attn_split_plan
+    wl = small_case("split_tail", 6, 128, (1200,), (2800, 300), 64, seed=91)
+    inp = make_inputs(wl)
+    layer, q, _, _ = place(wl, inp, fill=float("nan"))
+    parts, tail = attn_split_plan(layer.desc, wl.heads, 0)
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert (parts, tail) == attn_split_plan(layer.desc, wl.heads, 0, 148)
+        assert tail > 0
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[1], q.shape[0], dtype=torch.float32, device=q.device)
+    layer.forward(q, out, lse=lse, splits=0)
+    assert check_status() == WF_OK
+    ref, ref_lse = oracle_of(wl, inp)
+    assert_parity(out.float().cpu().numpy(), ref, f"{wl.name} plan ({parts}, {tail})")
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=2e-3)
+

@@ -3,7 +3,7 @@
 Collected last on purpose: it exercises the device-wide scratch array after every other test.
 The entry point must give exactly what wf_attn_forward_split gives with a caller workspace, on
 two calls in a row (the second reuses the scratch the first left behind), and must reject plans
-larger than its 96 MiB."""
+larger than its 128 MiB."""
 import ctypes
 
 import pytest
@@ -14,7 +14,7 @@ from block_causal_streaming_b200 import (WF_ERR_CAPACITY, WF_ERR_INVALID_ARG, WF
                                          check_status)
 from block_causal_streaming_b200.workloads import WP_RANK0, make_inputs, small_case
 
-SCRATCH_BYTES = 96 << 20
+SCRATCH_BYTES = 128 << 20
 FAKE = 0x10000
 
 
