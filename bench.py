@@ -28,6 +28,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -97,10 +98,15 @@ def workload_config(wl: Workload, world: int, split: bool) -> dict:
 
 
 def kernel_hash() -> str:
+    """Hash of the attention sources' code: comments and blank space removed, so that an edit of
+    a comment keeps a traffic record valid and any change of code drops it."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)       # block comments
+        text = re.sub(r"//[^\n]*", " ", text)                     # line comments
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

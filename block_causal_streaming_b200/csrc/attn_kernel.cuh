@@ -19,10 +19,15 @@
 //   warps 4-7  softmax of Q tile 1
 //   warp  8    TMA producer of Q (once) and of K_j (128 keys each) into the K ring, page by page
 //              through the page table; allocates/frees TMEM
-//   warp 11    TMA producer of V_j into the V ring; zeroes the rows of the last V tile past
-//              the last visible key
 //   warp  9    QK^T issuer (one thread): S_q = Q_q K_j^T (SS form)
 //   warp 10    P.V issuer (one thread): O_q += P_q V_j (TS form, P in TMEM)
+//   warp 11    TMA producer of V_j into the V ring; zeroes the rows of the last V tile past
+//              the last visible key
+// Two issuing threads because one thread's chain of MMAs into one accumulator runs well below
+// the tensor core's rate, and two independent chains in flight reach it; two producers because
+// the P.V thread trails the QK^T thread by the softmax, so V slots are held longer than K slots.
+// With key splits a unit runs as several CTAs, each over a consecutive part of its key tiles
+// (AttnParams::n_splits, n_tail).
 // TMEM (512 columns): one S buffer at [0, 128) that the two Q tiles take turns in (128 fp32
 // columns), P_q at [128 + 64 q, 192 + 64 q) (bf16 pairs) and O_q at [256 + D q, 256 + D q + D).
 //
