@@ -347,24 +347,27 @@ def fp8_kv_leg(wl: Workload, layer, k, v, dev, stream, steps: int, warmup: int,
 
 
 def int8_leg(wl: Workload, layer, q, dev, stream, steps: int, warmup: int, peak: float,
-             out_bf16) -> dict:
-    """The INT8 attention tier on the workload's layer: wf_qk_quantize_i8 (key mean, int8 codes
-    and scales of K' and Q) and wf_attn_forward_i8, each timed with CUDA events on the launching
-    stream; TFLOP/s on the same algorithmic FLOP count as the bf16 path.  `out_bf16`: the bf16
-    path's output, for the tier's deviation from it."""
+             out_bf16, fmt: str = "int8") -> dict:
+    """An 8-bit QK^T attention tier on the workload's layer -- fmt "int8": wf_qk_quantize_i8 (key
+    mean, int8 codes and scales of K' and Q) and wf_attn_forward_i8; "e4m3": wf_qk_quantize_e4m3
+    and wf_attn_forward_e4m3 -- each timed with CUDA events on the launching stream; TFLOP/s on
+    the same algorithmic FLOP count as the bf16 path.  `out_bf16`: the bf16 path's output, for
+    the tier's deviation from it."""
     import block_causal_streaming_b200 as wf
-    from block_causal_streaming_b200.layer import QkI8Buffers
-    qk = QkI8Buffers(layer.desc, wl.heads, wl.head_dim, dev)
+    from block_causal_streaming_b200.layer import QkE4m3Buffers, QkI8Buffers
+    e4m3 = fmt == "e4m3"
+    qk = (QkE4m3Buffers if e4m3 else QkI8Buffers)(layer.desc, wl.heads, wl.head_dim, dev)
     out = torch.empty_like(q)
     row = layer.page_tables[layer.layer]
     scale = 1.0 / np.sqrt(wl.head_dim)
+    quantize = wf.qk_quantize_e4m3 if e4m3 else wf.qk_quantize_i8
+    forward = wf.attn_forward_e4m3 if e4m3 else wf.attn_forward_i8
 
     def quant():
-        wf.qk_quantize_i8(q, layer.pool.k, layer.pool.v, row, layer.desc, qk, stream)
+        quantize(q, layer.pool.k, layer.pool.v, row, layer.desc, qk, stream)
 
     def attn():
-        wf.attn_forward_i8(qk, layer.pool.k, layer.pool.v, row, layer.desc, scale, out,
-                           None, stream)
+        forward(qk, layer.pool.k, layer.pool.v, row, layer.desc, scale, out, None, stream)
 
     for _ in range(warmup):
         quant()
@@ -380,7 +383,7 @@ def int8_leg(wl: Workload, layer, q, dev, stream, steps: int, warmup: int, peak:
     torch.cuda.synchronize(dev)
     rc = wf.check_status()
     if rc != wf.WF_OK:
-        raise RuntimeError(f"device status after the INT8 leg: {wf.strerror(rc)}")
+        raise RuntimeError(f"device status after the {fmt} leg: {wf.strerror(rc)}")
     q_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     a_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     flop = attention_flops(wl)
@@ -553,14 +556,17 @@ def gpu_arm(args, world, rank, local):
     if args.fp8_kv:
         res["fp8_kv"] = fp8_kv_leg(wl, layer, k, v, dev, stream, max(5, min(args.steps, 20)),
                                    args.warmup, float(peaks["hbm_gbs"]))
-    if args.int8:
-        if D != 128:
-            res["int8"] = {"unavailable": "the INT8 tier runs head_dim 128"}
-        else:
-            ref_out = torch.empty_like(q)
-            layer.forward(q, ref_out, scale=scale)
-            res["int8"] = int8_leg(wl, layer, q, dev, stream, max(5, min(args.steps, 20)),
-                                   args.warmup, peak, ref_out)
+    if args.int8 or args.e4m3:
+        ref_out = torch.empty_like(q)
+        layer.forward(q, ref_out, scale=scale)
+        for fmt, on in (("int8", args.int8), ("e4m3", args.e4m3)):
+            if not on:
+                continue
+            if D != 128:
+                res[fmt] = {"unavailable": "the 8-bit tiers run head_dim 128"}
+            else:
+                res[fmt] = int8_leg(wl, layer, q, dev, stream, max(5, min(args.steps, 20)),
+                                    args.warmup, peak, ref_out, fmt)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         tflops, info = oracle_sample(wl, inp, target_s=args.cpu_seconds)
         res["cpu_baseline"] = {"value": round(tflops, 6), "unit": UNIT,
@@ -620,6 +626,8 @@ def main(argv=None):
     ap.add_argument("--int8", action="store_true",
                     help="also time the INT8 attention tier (quantize + attention) on the "
                          "workload's layer")
+    ap.add_argument("--e4m3", action="store_true",
+                    help="also time the FP8 (e4m3) attention tier (quantize + attention)")
     ap.add_argument("--fp8-kv", action="store_true",
                     help="also time the FP8 K/V transport kernels (append to e4m3 pages, "
                          "dequantize) on the workload's chunks")

@@ -15,7 +15,9 @@ The product is the C-ABI library ``libwf_b200.so`` (declared in ``include/wf.h``
   ``wf_kv_append_publish_fp8`` / ``wf_kv_dequant_published`` publish those codes into other GPUs'
   FP8 pools with a generation flag, and convert a published chunk once its flag is up;
 * ``wf_qk_quantize_i8`` / ``wf_attn_forward_i8`` -- the INT8 tier: smoothed int8 K and int8 Q
-  with per-128-row scales, QK^T as an integer product on the tensor core.
+  with per-128-row scales, QK^T as an integer product on the tensor core;
+  ``wf_qk_quantize_e4m3`` / ``wf_attn_forward_e4m3`` the FP8 tier: e4m3 Q and K with
+  per-128-row scales, QK^T on the tensor core's 8-bit floating format.
 
 This package is its thin Python binding (ctypes, argument marshalling only), a small helper that
 owns the paged pools of one layer (:mod:`.layer`), the round-by-round planner of a streaming
@@ -30,7 +32,8 @@ _ABI_NAMES = (
     "selftest_timeout", "attn_forward_split", "attn_workspace_size",
     "attn_forward_split_noalloc", "kv_append_publish", "attn_forward_published", "ipc_export",
     "ipc_import", "ipc_close", "PoolDst", "kv_append_fp8", "kv_dequant", "KvPoolFp8",
-    "kv_append_fp8_chunks", "kv_dequant_chunks", "attn_split_plan",
+    "kv_append_fp8_chunks", "kv_dequant_chunks", "attn_split_plan", "qk_e4m3_sizes",
+    "qk_quantize_e4m3", "attn_forward_e4m3", "QkE4m3",
     "kv_append_publish_fp8", "kv_dequant_published", "Fp8Dst", "qk_i8_sizes", "qk_quantize_i8",
     "attn_forward_i8", "QkI8", "Segments", "attn_forward_segments",
     "attn_segments_workspace_size",

@@ -30,7 +30,8 @@ EXPORTED = ("wf_kv_append", "wf_attn_forward", "wf_check_status", "wf_strerror",
             "wf_attn_forward_split_noalloc", "wf_kv_append_publish", "wf_attn_forward_published",
             "wf_ipc_export", "wf_ipc_import", "wf_ipc_close", "wf_kv_append_fp8",
             "wf_kv_dequant", "wf_kv_append_fp8_chunks", "wf_kv_dequant_chunks",
-            "wf_attn_split_plan", "wf_kv_append_publish_fp8", "wf_kv_dequant_published",
+            "wf_attn_split_plan", "wf_qk_e4m3_sizes", "wf_qk_quantize_e4m3",
+            "wf_attn_forward_e4m3", "wf_kv_append_publish_fp8", "wf_kv_dequant_published",
             "wf_qk_i8_sizes", "wf_qk_quantize_i8", "wf_attn_forward_i8",
             "wf_attn_forward_segments", "wf_attn_segments_workspace_size",
             "wf_window_slots", "wf_window_round", "wf_window_round_ring")
@@ -60,6 +61,12 @@ class QkI8(ctypes.Structure):
     _fields_ = [("q_codes", ctypes.c_void_p), ("q_scale", ctypes.c_void_p),
                 ("k_codes", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
                 ("k_mean", ctypes.c_void_p), ("k_sum", ctypes.c_void_p)]
+
+
+class QkE4m3(ctypes.Structure):
+    """wf_qk_e4m3_t: the e4m3 Q and K of the FP8 tier (device pointers)."""
+    _fields_ = [("q_codes", ctypes.c_void_p), ("q_scale", ctypes.c_void_p),
+                ("k_codes", ctypes.c_void_p), ("k_scale", ctypes.c_void_p)]
 
 
 class KvPool(ctypes.Structure):
@@ -193,6 +200,18 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
                                        ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(Wavefront),
                                        f32, vp, ctypes.POINTER(ctypes.c_float), vp]
     lib.wf_attn_forward_i8.restype = i32
+    lib.wf_qk_e4m3_sizes.argtypes = [ctypes.POINTER(Wavefront), i32, i32,
+                                     ctypes.POINTER(ctypes.c_size_t)]
+    lib.wf_qk_e4m3_sizes.restype = i32
+    lib.wf_qk_quantize_e4m3.argtypes = [vp, ctypes.POINTER(KvPool),
+                                        ctypes.POINTER(ctypes.c_int32),
+                                        ctypes.POINTER(Wavefront), ctypes.POINTER(QkE4m3), vp]
+    lib.wf_qk_quantize_e4m3.restype = i32
+    lib.wf_attn_forward_e4m3.argtypes = [ctypes.POINTER(QkE4m3), ctypes.POINTER(KvPool),
+                                         ctypes.POINTER(ctypes.c_int32),
+                                         ctypes.POINTER(Wavefront), f32, vp,
+                                         ctypes.POINTER(ctypes.c_float), vp]
+    lib.wf_attn_forward_e4m3.restype = i32
     lib.wf_window_slots.argtypes = [ctypes.POINTER(WindowC), ctypes.POINTER(ctypes.c_int32),
                                     ctypes.POINTER(ctypes.c_int64)]
     lib.wf_window_slots.restype = i32
@@ -646,6 +665,77 @@ def attn_forward_i8(qk, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale
                                 _stream_handle(stream))
     if rc != WF_OK:
         raise WfError(rc, "wf_attn_forward_i8")
+
+
+QK_E4M3_FIELDS = ("q_codes", "q_scale", "k_codes", "k_scale")
+
+
+def qk_e4m3_sizes(wf: WavefrontDesc, num_heads: int, head_dim: int):
+    """wf_qk_e4m3_sizes: byte sizes of the four buffers of the FP8 tier, in QK_E4M3_FIELDS
+    order."""
+    sizes = (ctypes.c_size_t * 4)()
+    rc = lib.wf_qk_e4m3_sizes(ctypes.byref(wf.c), int(num_heads), int(head_dim), sizes)
+    if rc != WF_OK:
+        raise WfError(rc, "wf_qk_e4m3_sizes")
+    return [int(x) for x in sizes]
+
+
+def _qk_e4m3_struct(qk) -> QkE4m3:
+    """qk: a mapping / object with the four QK_E4M3_FIELDS device tensors (codes uint8)."""
+    get = (lambda n: qk[n]) if isinstance(qk, dict) else (lambda n: getattr(qk, n))
+    for n, d in zip(QK_E4M3_FIELDS, ("u8", "f32", "u8", "f32")):
+        _check_tensor(get(n), n, d)
+    return QkE4m3(*[get(n).data_ptr() for n in QK_E4M3_FIELDS])
+
+
+def qk_quantize_e4m3(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, qk,
+                     stream=None) -> None:
+    """wf_qk_quantize_e4m3: e4m3 Q (from q) and K (from the K pool) with their scales into qk."""
+    _, _, H, D = _pool_shape(k_pool, v_pool)
+    _check_queries(q, q, None, wf, H, D)
+    _check_page_table_row(page_table_row, wf)
+    sizes = qk_e4m3_sizes(wf, H, D)
+    get = (lambda n: qk[n]) if isinstance(qk, dict) else (lambda n: getattr(qk, n))
+    for n, sz in zip(QK_E4M3_FIELDS, sizes):
+        t = get(n)
+        if t.numel() * t.element_size() < sz:
+            raise ValueError(f"{n}: {t.numel() * t.element_size()} bytes, needs {sz}")
+    for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"),
+                    (page_table_row, "page_table_row", "i32")):
+        _check_tensor(t, n, d)
+    pool = _pool_struct(k_pool, v_pool)
+    s = _qk_e4m3_struct(qk)
+    rc = lib.wf_qk_quantize_e4m3(q.data_ptr(), ctypes.byref(pool),
+                                 ctypes.cast(ctypes.c_void_p(page_table_row.data_ptr()),
+                                             ctypes.POINTER(ctypes.c_int32)),
+                                 ctypes.byref(wf.c), ctypes.byref(s), _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_qk_quantize_e4m3")
+
+
+def attn_forward_e4m3(qk, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: float, out,
+                      lse=None, stream=None) -> None:
+    """wf_attn_forward_e4m3: block-causal attention on the e4m3 Q / K of qk, V from v_pool."""
+    _, _, H, D = _pool_shape(k_pool, v_pool)
+    _check_queries(out, out, lse, wf, H, D)
+    _check_page_table_row(page_table_row, wf)
+    for t, n, d in ((out, "out", "bf16"), (v_pool, "v_pool", "bf16"),
+                    (page_table_row, "page_table_row", "i32")):
+        _check_tensor(t, n, d)
+    if lse is not None:
+        _check_tensor(lse, "lse", "f32")
+    pool = _pool_struct(k_pool, v_pool)
+    s = _qk_e4m3_struct(qk)
+    rc = lib.wf_attn_forward_e4m3(ctypes.byref(s), ctypes.byref(pool),
+                                  ctypes.cast(ctypes.c_void_p(page_table_row.data_ptr()),
+                                              ctypes.POINTER(ctypes.c_int32)),
+                                  ctypes.byref(wf.c), float(scale), out.data_ptr(),
+                                  ctypes.cast(ctypes.c_void_p(lse.data_ptr()),
+                                              ctypes.POINTER(ctypes.c_float))
+                                  if lse is not None else None,
+                                  _stream_handle(stream))
+    if rc != WF_OK:
+        raise WfError(rc, "wf_attn_forward_e4m3")
 
 
 def attn_forward(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale: float, out,

@@ -188,10 +188,13 @@ struct AttnSmem {
 // loading their keys; a separate instantiation so the plain kernel carries none of that code.
 // kI8: the INT8 tier -- S = Q_i8 K_i8^T on the tensor core (kind::i8, s32 in TMEM), each S tile
 // scaled by scale_q x scale_k in the softmax; P and P.V as in the bf16 kernel.
-template <int D, bool kWaitPublished = false, bool kI8 = false>
+// kE4M3 (with kI8): the FP8 tier -- the 8-bit Q and K codes are e4m3, S = Q K^T by kind::f8f6f4
+// with fp32 accumulation; scales, P and P.V as in the INT8 tier.
+template <int D, bool kWaitPublished = false, bool kI8 = false, bool kE4M3 = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     wf_attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   static_assert(!kI8 || (D == 128 && !kWaitPublished), "the INT8 tier runs head_dim 128");
+  static_assert(!kE4M3 || kI8, "the FP8 tier is an 8-bit tier");
   using L = AttnSmem<D, kI8>;
   constexpr int BN = L::BN, DH = L::DH, NS = L::NS;
   constexpr uint32_t QTILE = L::QTILE, QHALF = L::QHALF, KTILE = L::KTILE, KHALF = L::KHALF;
@@ -291,7 +294,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(L::B_SF));
-          if (kI8) {
+          if (kI8 && !kE4M3) {
             // s32 -> fp32, exact: |S| <= 128 x 127^2 < 2^24.  (Reading the bits of
             // 1.5 x 2^23 + S as a float and subtracting 1.5 x 2^23 measured 3 % slower.)
   #pragma unroll
@@ -533,8 +536,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // rate; two independent chains in flight together run at the full rate.  Descriptors are
       // built once; per instruction only a compile-time offset (16-byte units) is added to the
       // start-address field, so the issue loop stays a few instructions per MMA.
-      constexpr uint32_t idesc_qk = kI8 ? idesc_s8_s32(kBM, BN)      // Q, K both K-major
-                                        : idesc_bf16_f32(kBM, BN, 0, 0);
+      constexpr uint32_t idesc_qk = kE4M3 ? idesc_e4m3_f32(kBM, BN)   // Q, K both K-major
+                                    : kI8 ? idesc_s8_s32(kBM, BN)
+                                          : idesc_bf16_f32(kBM, BN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);     // P (TMEM), V MN-major
       const uint64_t dq0 = smem_desc_sw128(base + L::Q_OFF, 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(base + L::KV_OFF, 16, 1024);
@@ -553,7 +557,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint64_t dq = dq0 + ((static_cast<uint32_t>(q) * QTILE) >> 4);
   #pragma unroll
           for (int kk = 0; kk < kSteps; ++kk) {
-            if (kI8)
+            if (kE4M3)
+              umma_ss_f8(tmem, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), idesc_qk,
+                         kk > 0 ? 1u : 0u);
+            else if (kI8)
               umma_ss_i8(tmem, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), idesc_qk,
                          kk > 0 ? 1u : 0u);
             else

@@ -23,6 +23,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include <cstdint>
 
@@ -86,9 +87,11 @@ __global__ void wf_kmean_finalize(const __grid_constant__ QkI8Params p, int cols
 }
 
 // One CTA per (block, head): 128 rows x D values, two threads per row (D / 2 values each).
-// kKeys: rows are logical keys read through the page table and smoothed by k_mean; else query
-// rows of q.
-template <int D, bool kKeys>
+// kKeys: rows are logical keys read through the page table (smoothed by k_mean for int8); else
+// query rows of q.  kE4M3: the FP8 tier's codes instead -- scale = amax / 448,
+// code = e4m3(x * (448 / amax)) rounded to nearest even and saturated (cvt.rn.satfinite), no
+// smoothing; the same block layout.
+template <int D, bool kKeys, bool kE4M3 = false>
 __global__ void __launch_bounds__(kQuantI8Threads)
     wf_block_quant_kernel(const __grid_constant__ QkI8Params p) {
   constexpr int HALF = D / 2;               // values per thread
@@ -120,7 +123,7 @@ __global__ void __launch_bounds__(kQuantI8Threads)
           x[8 * i + 2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
         }
       }
-      if (kKeys) {
+      if (kKeys && !kE4M3) {
         const float* mu = p.k_mean + h * D + half * HALF;
 #pragma unroll
         for (int i = 0; i < HALF; ++i) x[i] = x[i] - __ldg(mu + i);
@@ -139,12 +142,13 @@ __global__ void __launch_bounds__(kQuantI8Threads)
   a = red[0];
 #pragma unroll
   for (int w = 1; w < kQuantI8Threads / 32; ++w) a = fmaxf(a, red[w]);
-  float inv = 127.0f / a;                     // IEEE division: these values decide codes
+  constexpr float kQmax = kE4M3 ? 448.0f : 127.0f;
+  float inv = kQmax / a;                      // IEEE division: these values decide codes
   const bool nz = a > 0.f && isfinite(inv);
   inv = nz ? inv : 0.f;
   if (threadIdx.x == 0) {
     const int nblocks = (rows + kI8Block - 1) / kI8Block;
-    (kKeys ? p.k_scale : p.q_scale)[h * nblocks + b] = nz ? a / 127.0f : 0.f;
+    (kKeys ? p.k_scale : p.q_scale)[h * nblocks + b] = nz ? a / kQmax : 0.f;
   }
   if (!live) return;
   int8_t* dst = (kKeys ? p.k_codes : p.q_codes) + static_cast<int64_t>(r) * cols + h * D +
@@ -155,11 +159,21 @@ __global__ void __launch_bounds__(kQuantI8Threads)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       uint32_t word = 0;
+      if (kE4M3) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        int c = __float2int_rn(x[16 * i + 4 * j + e] * inv);   // round half to even
-        c = max(-127, min(127, c));
-        word |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * e);
+        for (int e = 0; e < 4; e += 2) {
+          const float2 y = make_float2(x[16 * i + 4 * j + e] * inv,
+                                       x[16 * i + 4 * j + e + 1] * inv);
+          const uint32_t two = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+          word |= (two & 0xFFFFu) << (8 * e);                   // .x in the low byte
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          int c = __float2int_rn(x[16 * i + 4 * j + e] * inv);   // round half to even
+          c = max(-127, min(127, c));
+          word |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * e);
+        }
       }
       w[j] = word;
     }

@@ -88,6 +88,9 @@ int device_state(DeviceState** out) {
                                  wfk::AttnSmem<64>::ALLOC) != cudaSuccess ||
             cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<128, false, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 wfk::AttnSmem<128, true>::ALLOC) != cudaSuccess ||
+            cudaFuncSetAttribute(wfk::wf_attn_fwd_kernel<128, false, true, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  wfk::AttnSmem<128, true>::ALLOC) != cudaSuccess) {
           cudaGetLastError();
           return WF_ERR_CUDA;
@@ -1211,32 +1214,114 @@ int wf_qk_quantize_i8(const void* q, const wf_kv_pool_t* kv_pages, const int32_t
   return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
-int wf_attn_forward_i8(const wf_qk_i8_t* qk, const wf_kv_pool_t* kv_pages,
-                       const int32_t* page_table_row, const wf_wavefront_t* wf, float scale,
-                       void* out, float* lse_or_null, wf_stream_t stream) {
-  if (qk == nullptr || qk->q_codes == nullptr || qk->k_codes == nullptr ||
-      qk->q_scale == nullptr || qk->k_scale == nullptr || !aligned16(qk->k_codes))
+}  // extern "C"
+
+namespace {
+
+// Attention over 8-bit Q and K codes with per-128-row scales (the INT8 or the FP8 tier).
+int attn_forward_8bit(void* q_codes, const float* q_scale, void* k_codes, const float* k_scale,
+                      bool e4m3, const wf_kv_pool_t* kv_pages, const int32_t* page_table_row,
+                      const wf_wavefront_t* wf, float scale, void* out, float* lse_or_null,
+                      wf_stream_t stream) {
+  if (q_codes == nullptr || k_codes == nullptr || q_scale == nullptr || k_scale == nullptr ||
+      !aligned16(k_codes))
     return WF_ERR_INVALID_ARG;
   if (kv_pages != nullptr && kv_pages->head_dim != 128) return WF_ERR_SHAPE;
   AttnLaunch L;
-  int rc = prepare_attention(qk->q_codes, kv_pages, page_table_row, wf, scale, out, lse_or_null,
-                             &L);
+  int rc = prepare_attention(q_codes, kv_pages, page_table_row, wf, scale, out, lse_or_null, &L);
   if (rc || L.p.T_q == 0) return rc;
   wfk::AttnParams& p = L.p;
   const int t_kv = wf->chunk_offsets[wf->num_chunks];
-  if (!encode_rows_u8(&p.tm_q, qk->q_codes, 128, p.H, p.T_q, wfk::kBM) ||
-      !encode_rows_u8(&p.tm_k, qk->k_codes, 128, p.H, t_kv, wfk::kBN))
+  if (!encode_rows_u8(&p.tm_q, q_codes, 128, p.H, p.T_q, wfk::kBM) ||
+      !encode_rows_u8(&p.tm_k, k_codes, 128, p.H, t_kv, wfk::kBN))
     return WF_ERR_CUDA;
-  p.q_scale = qk->q_scale;
-  p.k_scale = qk->k_scale;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
   p.nqt = (p.T_q + wfk::kBM - 1) / wfk::kBM;
   p.nkb = (t_kv + wfk::kBN - 1) / wfk::kBN;
   p.launch_id = g_launch_counter.fetch_add(1);
   if (p.launch_id == 0) p.launch_id = g_launch_counter.fetch_add(1);
   const unsigned g = static_cast<unsigned>(static_cast<int64_t>(p.n_pairs) * p.H);
-  wfk::wf_attn_fwd_kernel<128, false, true>
-      <<<g, wfk::kAttnThreads, wfk::AttnSmem<128, true>::ALLOC,
-         reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (e4m3)
+    wfk::wf_attn_fwd_kernel<128, false, true, true>
+        <<<g, wfk::kAttnThreads, wfk::AttnSmem<128, true>::ALLOC, s>>>(p);
+  else
+    wfk::wf_attn_fwd_kernel<128, false, true>
+        <<<g, wfk::kAttnThreads, wfk::AttnSmem<128, true>::ALLOC, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int wf_attn_forward_i8(const wf_qk_i8_t* qk, const wf_kv_pool_t* kv_pages,
+                       const int32_t* page_table_row, const wf_wavefront_t* wf, float scale,
+                       void* out, float* lse_or_null, wf_stream_t stream) {
+  if (qk == nullptr) return WF_ERR_INVALID_ARG;
+  return attn_forward_8bit(qk->q_codes, qk->q_scale, qk->k_codes, qk->k_scale, false, kv_pages,
+                           page_table_row, wf, scale, out, lse_or_null, stream);
+}
+
+int wf_attn_forward_e4m3(const wf_qk_e4m3_t* qk, const wf_kv_pool_t* kv_pages,
+                         const int32_t* page_table_row, const wf_wavefront_t* wf, float scale,
+                         void* out, float* lse_or_null, wf_stream_t stream) {
+  if (qk == nullptr) return WF_ERR_INVALID_ARG;
+  return attn_forward_8bit(qk->q_codes, qk->q_scale, qk->k_codes, qk->k_scale, true, kv_pages,
+                           page_table_row, wf, scale, out, lse_or_null, stream);
+}
+
+int wf_qk_e4m3_sizes(const wf_wavefront_t* wf, int num_heads, int head_dim, size_t sizes[4]) {
+  size_t all[6];
+  const int rc = wf_qk_i8_sizes(wf, num_heads, head_dim, all);
+  if (rc) return rc;
+  for (int i = 0; i < 4; ++i) sizes[i] = all[i];
+  return WF_OK;
+}
+
+int wf_qk_quantize_e4m3(const void* q, const wf_kv_pool_t* kv_pages,
+                        const int32_t* page_table_row, const wf_wavefront_t* wf,
+                        const wf_qk_e4m3_t* qk, wf_stream_t stream) {
+  int rc = validate_pool(kv_pages);
+  if (rc) return rc;
+  if (kv_pages->head_dim != 128) return WF_ERR_SHAPE;
+  int t_kv = 0;
+  rc = validate_wavefront(wf, kv_pages, &t_kv);
+  if (rc) return rc;
+  if (wf->num_ctx_chunks >= wf->num_chunks) return WF_ERR_SHAPE;
+  const int t_q = t_kv - wf->chunk_offsets[wf->num_ctx_chunks];
+  if (t_q == 0) return WF_OK;
+  if (q == nullptr || qk == nullptr || page_table_row == nullptr || !aligned16(q) ||
+      qk->q_codes == nullptr || qk->k_codes == nullptr || qk->q_scale == nullptr ||
+      qk->k_scale == nullptr || !aligned16(qk->q_codes) || !aligned16(qk->k_codes) ||
+      (reinterpret_cast<uintptr_t>(qk->q_scale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(qk->k_scale) & 3u))
+    return WF_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  rc = device_state(&d);
+  if (rc) return rc;
+  const int H = kv_pages->num_heads;
+  wfk::QkI8Params p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_pool = static_cast<const __nv_bfloat16*>(kv_pages->k_pool);
+  p.pt_row = page_table_row;
+  p.q_codes = static_cast<int8_t*>(qk->q_codes);
+  p.q_scale = qk->q_scale;
+  p.k_codes = static_cast<int8_t*>(qk->k_codes);
+  p.k_scale = qk->k_scale;
+  p.status = d->status;
+  p.T_q = t_q;
+  p.T_kv = t_kv;
+  p.H = H;
+  p.page_size = kv_pages->page_size;
+  p.num_pages = kv_pages->num_pages;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  wfk::wf_block_quant_kernel<128, true, true>
+      <<<dim3((t_kv + wfk::kI8Block - 1) / wfk::kI8Block, H), wfk::kQuantI8Threads, 0, s>>>(p);
+  wfk::wf_block_quant_kernel<128, false, true>
+      <<<dim3((t_q + wfk::kI8Block - 1) / wfk::kI8Block, H), wfk::kQuantI8Threads, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 

@@ -66,6 +66,22 @@ class QkI8Buffers:
         self.heads = heads
 
 
+class QkE4m3Buffers:
+    """The device buffers of the FP8 (e4m3) attention tier for one wavefront shape (see
+    ``wf_qk_quantize_e4m3``): e4m3 Q and K codes (uint8) and their per-128-row scales."""
+
+    def __init__(self, desc, heads: int, head_dim: int, device="cuda"):
+        from . import _abi
+        sizes = _abi.qk_e4m3_sizes(desc, heads, head_dim)
+        off = desc.chunk_offsets
+        t_kv, t_q = off[-1], off[-1] - off[desc.num_ctx_chunks]
+        self.q_codes = torch.empty(t_q, heads, head_dim, dtype=torch.uint8, device=device)
+        self.q_scale = torch.empty(sizes[1] // 4, dtype=torch.float32, device=device)
+        self.k_codes = torch.empty(t_kv, heads, head_dim, dtype=torch.uint8, device=device)
+        self.k_scale = torch.empty(sizes[3] // 4, dtype=torch.float32, device=device)
+        self.heads = heads
+
+
 class WavefrontLayer:
     """One layer of a wavefront: its descriptor and its page-table rows.
 
@@ -112,6 +128,18 @@ class WavefrontLayer:
         _abi.qk_quantize_i8(q, self.pool.k, self.pool.v, row, self.desc, qk, stream)
         _abi.attn_forward_i8(qk, self.pool.k, self.pool.v, row, self.desc, scale, out, lse,
                              stream)
+
+    def forward_e4m3(self, q: torch.Tensor, out: torch.Tensor, qk: "QkE4m3Buffers",
+                     scale: Optional[float] = None, lse: Optional[torch.Tensor] = None,
+                     stream=None) -> None:
+        """The FP8 tier: quantize q and this layer's keys into ``qk`` as e4m3, then attend."""
+        from . import _abi
+        if scale is None:
+            scale = 1.0 / math.sqrt(self.pool.head_dim)
+        row = self.page_tables[self.layer]
+        _abi.qk_quantize_e4m3(q, self.pool.k, self.pool.v, row, self.desc, qk, stream)
+        _abi.attn_forward_e4m3(qk, self.pool.k, self.pool.v, row, self.desc, scale, out, lse,
+                               stream)
 
     def forward(self, q: torch.Tensor, out: torch.Tensor, scale: Optional[float] = None,
                 lse: Optional[torch.Tensor] = None, stream=None,

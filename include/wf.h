@@ -426,6 +426,44 @@ int wf_attn_forward_i8(const wf_qk_i8_t* qk, const wf_kv_pool_t* kv_pages,
                        const int32_t* page_table_row, const wf_wavefront_t* wf, float scale,
                        void* out, float* lse_or_null, wf_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * FP8 (e4m3) attention tier: the e4m3 twin of the INT8 tier, QK^T on tcgen05.mma kind::f8f6f4
+ * (project page, "03 End-to-end KV transport", item 01 "Precision", measures K/V in FP8; the
+ * pages give no scale granularity for attention operands, so the blocks are the INT8 tier's).
+ *   wf_qk_quantize_e4m3  Q per (128 query rows, head) and K per (128 keys, head), counted from
+ *                        row / key 0, as e4m3 codes with scale = amax / 448:
+ *                        code = e4m3(x * (448 / amax)), fp32 steps, rounded to nearest even and
+ *                        saturated at 448 (a block of zeros, or one whose 448 / amax overflows,
+ *                        gets scale 0); no key smoothing.
+ *   wf_attn_forward_e4m3 the block-causal attention of wf_attn_forward with
+ *                        S = scale * scale_q * scale_k * (Q_e4m3 . K_e4m3), fp32 accumulation on
+ *                        the tensor core, and P.V in bf16 over the unquantized V pages.
+ * Head dimension 128 only (WF_ERR_SHAPE otherwise).  Buffers as the INT8 tier's first four, with
+ * e4m3 codes (one byte each) in place of int8; sizes from wf_qk_e4m3_sizes.
+ * --------------------------------------------------------------------------------------------- */
+typedef struct {
+  void* q_codes;      /* e4m3 [T_q][H][128], 16-byte aligned */
+  float* q_scale;     /* fp32 [H][ceil(T_q / 128)] */
+  void* k_codes;      /* e4m3 [T_kv][H][128], logical key order, 16-byte aligned */
+  float* k_scale;     /* fp32 [H][ceil(T_kv / 128)] */
+} wf_qk_e4m3_t;
+
+/* Byte sizes of the four wf_qk_e4m3_t buffers, in field order.  WF_ERR_SHAPE unless head_dim is
+ * 128. */
+int wf_qk_e4m3_sizes(const wf_wavefront_t* wf, int num_heads, int head_dim, size_t sizes[4]);
+
+/* Quantize q (bf16 [T_q][H][128]) and the layer's keys (the K pool through page_table_row, all
+ * T_kv tokens) into `qk`.  Errors as wf_qk_quantize_i8.  Asynchronous on `stream`. */
+int wf_qk_quantize_e4m3(const void* q, const wf_kv_pool_t* kv_pages,
+                        const int32_t* page_table_row, const wf_wavefront_t* wf,
+                        const wf_qk_e4m3_t* qk, wf_stream_t stream);
+
+/* wf_attn_forward on e4m3 Q and K (filled by wf_qk_quantize_e4m3 for the same wavefront and page
+ * table); V is read from kv_pages.  out, lse_or_null and errors as wf_attn_forward. */
+int wf_attn_forward_e4m3(const wf_qk_e4m3_t* qk, const wf_kv_pool_t* kv_pages,
+                         const int32_t* page_table_row, const wf_wavefront_t* wf, float scale,
+                         void* out, float* lse_or_null, wf_stream_t stream);
+
 /*
  * Rolling context window: the plan of one round of a stream (host only, no device work).
  *
