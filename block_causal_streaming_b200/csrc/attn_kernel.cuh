@@ -121,8 +121,9 @@ struct AttnParams {
   unsigned flag_gen;
   int nchunks;
   int chunk_end[kMaxQChunks];
-  // INT8 tier (kI8): tm_q / tm_k describe int8 Q and K' codes ([rows][H][D], K' contiguous in
-  // logical key order), with one scale per (128 rows, head): q_scale [H][nqt], k_scale [H][nkb].
+  // 8-bit tiers (kI8; kE4M3 for e4m3): tm_q / tm_k describe the 8-bit Q and K codes
+  // ([rows][H][D], K contiguous in logical key order), with one scale per (128 rows, head):
+  // q_scale [H][nqt], k_scale [H][nkb].
   const float* q_scale;
   const float* k_scale;
   int nqt, nkb;
@@ -155,8 +156,8 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-// kI8: Q and K tiles hold int8 codes (one 128-byte row per query / key at head_dim 128), V
-// stays bf16; the 32 KB Q saves go to a sixth ring slot.
+// kI8: Q and K tiles hold 8-bit codes (int8 or e4m3; one 128-byte row per query / key at
+// head_dim 128), V stays bf16; the 32 KB Q saves go to a sixth ring slot.
 template <int D, bool kI8 = false>
 struct AttnSmem {
   static constexpr int BN = kBN;

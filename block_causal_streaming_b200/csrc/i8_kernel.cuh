@@ -1,4 +1,5 @@
-// i8_kernel.cuh -- quantization of Q and K for the INT8 (Sage-like) attention tier (sm_100a).
+// i8_kernel.cuh -- quantization of Q and K for the 8-bit attention tiers (sm_100a): INT8
+// (Sage-like) and FP8 (e4m3).
 //
 // The pages name SageAttention with W8A8 as the fast attention backend (GitHub README, results
 // table, "Sage . causal . paged" rows; KipQuest abstract) and give no internals.  The tier built
@@ -14,12 +15,17 @@
 //     code = clamp(round_half_even(x * inv), -127, 127) with an fp32 product.
 // The blocks are the attention kernel's Q tiles and K tiles, so each S tile is dequantized by one
 // scalar (scale_q x scale_k) folded into the softmax's existing multiply.
+// The FP8 tier (project page, "03 End-to-end KV transport", item 01 "Precision", measures K/V in
+// FP8; the pages give no granularity for attention operands) uses the same blocks without the key
+// mean: inv = 448 / a, scale = a / 448, code = e4m3(x * inv) rounded to nearest even and
+// saturated (the FP8 K/V pages' encoder).
 //
 // Kernels:
 //   wf_kmean_kernel     fp64 column sums of the paged bf16 keys (atomics into k_sum, zeroed first)
 //   wf_kmean_finalize   k_mean = fp32(k_sum / T_kv)
-//   wf_block_quant_kernel<kKeys>  one CTA per (block, head): K' (through the page table) or Q,
-//                       largest magnitude, codes into a contiguous int8 [rows][H][D] and the scale.
+//   wf_block_quant_kernel<kKeys, kE4M3>  one CTA per (block, head): K' (through the page table)
+//                       or Q, largest magnitude, codes into a contiguous [rows][H][D] (int8 or
+//                       e4m3) and the scale.
 #pragma once
 
 #include <cuda_bf16.h>
