@@ -327,6 +327,16 @@ def _check_tensor(t, name: str, dtype_name: str):
         raise ValueError(f"{name}: expected a contiguous tensor")
 
 
+def _check_qk_buffers(qk, fields, sizes):
+    """Every buffer of an 8-bit tier's qk holds at least the bytes the library's sizes call
+    gives for this wavefront (the quantize call writes them all, the attention call reads them)."""
+    get = (lambda n: qk[n]) if isinstance(qk, dict) else (lambda n: getattr(qk, n))
+    for n, sz in zip(fields, sizes):
+        t = get(n)
+        if t.numel() * t.element_size() < sz:
+            raise ValueError(f"{n}: {t.numel() * t.element_size()} bytes, needs {sz}")
+
+
 class Window:
     """Host copy of a wf_window_t; keeps the stage array alive while C reads it."""
 
@@ -623,12 +633,7 @@ def qk_quantize_i8(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, qk,
     _, _, H, D = _pool_shape(k_pool, v_pool)
     _check_queries(q, q, None, wf, H, D)
     _check_page_table_row(page_table_row, wf)
-    sizes = qk_i8_sizes(wf, H, D)
-    get = (lambda n: qk[n]) if isinstance(qk, dict) else (lambda n: getattr(qk, n))
-    for n, sz in zip(QK_I8_FIELDS, sizes):
-        t = get(n)
-        if t.numel() * t.element_size() < sz:
-            raise ValueError(f"{n}: {t.numel() * t.element_size()} bytes, needs {sz}")
+    _check_qk_buffers(qk, QK_I8_FIELDS, qk_i8_sizes(wf, H, D))
     for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"),
                     (page_table_row, "page_table_row", "i32")):
         _check_tensor(t, n, d)
@@ -648,6 +653,7 @@ def attn_forward_i8(qk, k_pool, v_pool, page_table_row, wf: WavefrontDesc, scale
     _, _, H, D = _pool_shape(k_pool, v_pool)
     _check_queries(out, out, lse, wf, H, D)
     _check_page_table_row(page_table_row, wf)
+    _check_qk_buffers(qk, QK_I8_FIELDS, qk_i8_sizes(wf, H, D))
     for t, n, d in ((out, "out", "bf16"), (v_pool, "v_pool", "bf16"),
                     (page_table_row, "page_table_row", "i32")):
         _check_tensor(t, n, d)
@@ -694,12 +700,7 @@ def qk_quantize_e4m3(q, k_pool, v_pool, page_table_row, wf: WavefrontDesc, qk,
     _, _, H, D = _pool_shape(k_pool, v_pool)
     _check_queries(q, q, None, wf, H, D)
     _check_page_table_row(page_table_row, wf)
-    sizes = qk_e4m3_sizes(wf, H, D)
-    get = (lambda n: qk[n]) if isinstance(qk, dict) else (lambda n: getattr(qk, n))
-    for n, sz in zip(QK_E4M3_FIELDS, sizes):
-        t = get(n)
-        if t.numel() * t.element_size() < sz:
-            raise ValueError(f"{n}: {t.numel() * t.element_size()} bytes, needs {sz}")
+    _check_qk_buffers(qk, QK_E4M3_FIELDS, qk_e4m3_sizes(wf, H, D))
     for t, n, d in ((q, "q", "bf16"), (k_pool, "k_pool", "bf16"),
                     (page_table_row, "page_table_row", "i32")):
         _check_tensor(t, n, d)
@@ -719,6 +720,7 @@ def attn_forward_e4m3(qk, k_pool, v_pool, page_table_row, wf: WavefrontDesc, sca
     _, _, H, D = _pool_shape(k_pool, v_pool)
     _check_queries(out, out, lse, wf, H, D)
     _check_page_table_row(page_table_row, wf)
+    _check_qk_buffers(qk, QK_E4M3_FIELDS, qk_e4m3_sizes(wf, H, D))
     for t, n, d in ((out, "out", "bf16"), (v_pool, "v_pool", "bf16"),
                     (page_table_row, "page_table_row", "i32")):
         _check_tensor(t, n, d)
