@@ -249,12 +249,14 @@ def oracle_sample(wl: Workload, inp, target_s: float, seed: int = 0):
     v32 = inp.v.float().numpy()
     scale = 1.0 / np.sqrt(wl.head_dim)
     H = wl.heads
+    threads = oracle.default_threads()
 
     def run(rows):
         rr = np.repeat(np.asarray(rows, dtype=np.int32), H)
         hh = np.tile(np.arange(H, dtype=np.int32), len(rows))
         t0 = time.perf_counter()
-        oracle.attention_rows(q32, k32, v32, wl.chunk_offsets, wl.num_ctx_chunks, scale, rr, hh)
+        oracle.attention_rows(q32, k32, v32, wl.chunk_offsets, wl.num_ctx_chunks, scale, rr, hh,
+                              nthreads=threads)
         return time.perf_counter() - t0
 
     probe = sorted(rng.choice(wl.t_q, size=4, replace=False).tolist())
@@ -264,7 +266,7 @@ def oracle_sample(wl: Workload, inp, target_s: float, seed: int = 0):
     rows = sorted(rng.choice(wl.t_q, size=n, replace=False).tolist())
     dt = run(rows)
     fl = rows_flops(wl, rows, H)
-    info = {"rows": n, "heads": H, "seconds": round(dt, 3), "flop": fl}
+    info = {"rows": n, "heads": H, "seconds": round(dt, 3), "flop": fl, "threads": threads}
     return fl / dt / 1e12, info
 
 
@@ -570,7 +572,7 @@ def gpu_arm(args, world, rank, local):
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         tflops, info = oracle_sample(wl, inp, target_s=args.cpu_seconds)
         res["cpu_baseline"] = {"value": round(tflops, 6), "unit": UNIT,
-                               "cores": os.cpu_count(), "kind": "oracle",
+                               "cores": info["threads"], "kind": "oracle",
                                "sample": f"{info['rows']} random query rows x {info['heads']} "
                                          f"heads of the same workload, {info['seconds']} s"}
     if world > 1:
@@ -589,9 +591,10 @@ def reference_arm(args, world, rank):
     per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
     for i in range(args.warmup):
         oracle_sample(wl, inp, target_s=min(per_step, 1.0), seed=1000 + i)
-    vals, secs, rows = [], 0.0, 0
+    vals, secs, rows, threads = [], 0.0, 0, 0
     for i in range(args.steps):
         v, info = oracle_sample(wl, inp, target_s=per_step, seed=i)
+        threads = info["threads"]
         vals.append(v)
         secs += info["seconds"]
         rows += info["rows"]
@@ -605,7 +608,7 @@ def reference_arm(args, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1)*0.5 bf16)", "impl": "reference",
         "config": workload_config(wl, world, wl is WP_RANK0),
-        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": os.cpu_count(),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},

@@ -101,8 +101,10 @@ def test_both_arms_print_the_same_config(monkeypatch):
         workload, steps, warmup, cpu_seconds = "wan13b_5step", 1, 3, 0.05
     monkeypatch.setattr(bench, "oracle_sample",
                         lambda wl, inp, target_s, seed=0: (1.0, {"rows": 4, "heads": wl.heads,
-                                                                 "seconds": 0.01, "flop": 1}))
+                                                                 "seconds": 0.01, "flop": 1,
+                                                                 "threads": 3}))
     line = bench.reference_arm(A, world=1, rank=0)
+    assert line["cpu_baseline"]["cores"] == 3          # the threads the oracle ran with
     assert line["config"] == bench.workload_config(WAN13B_5STEP, 1, False)
     assert line["config"]["chunks"] == "2 ctx + 5 active x 4680"
     assert "633 MB" in line["config"]["l2"]
