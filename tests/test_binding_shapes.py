@@ -73,7 +73,15 @@ def test_the_helpers_valid_calls_pass(fake):
         _abi.kv_append_fp8(*fp.tensors, 0, c, _kv(OFF[c + 1] - OFF[c]), _kv(OFF[c + 1] - OFF[c]),
                            lay.page_tables, lay.desc)
         _abi.kv_dequant(*fp.tensors, lay.pool.k, lay.pool.v, 0, c, lay.page_tables, lay.desc)
+    _abi.kv_append_fp8_chunks(*fp.tensors, 0, 0, 3, _kv(130), _kv(130), lay.page_tables, lay.desc)
+    _abi.kv_append_fp8_chunks(*fp.tensors, 0, 1, 3, _kv(90), _kv(90), lay.page_tables, lay.desc)
+    _abi.kv_dequant_chunks(*fp.tensors, lay.pool.k, lay.pool.v, 0, 0, 3, lay.page_tables,
+                           lay.desc)
     flags = torch.zeros(2, _abi.WF_MAX_CHUNKS, dtype=torch.int32)
+    _abi.kv_append_publish_fp8(*fp.tensors, flags, [], 0, 1, _kv(50), _kv(50), lay.page_tables,
+                               lay.desc, 2)
+    _abi.kv_dequant_published(*fp.tensors, lay.pool.k, lay.pool.v, 0, 1, lay.page_tables,
+                              lay.desc, flags[0], 2)
     pt2 = torch.stack([lay.page_tables[0], lay.page_tables[0]]).contiguous()
     _abi.kv_append_publish(lay.pool.k, lay.pool.v, flags, [], 1, 2, _kv(40), _kv(40), pt2,
                            lay.desc, 3)
@@ -89,12 +97,16 @@ def test_the_helpers_valid_calls_pass(fake):
         for layer in range(2):
             cache.run_layer(v, layer, _kv(rows), _kv(rows), _kv(rows), _kv(rows))
     assert "wf_attn_forward" in fake.calls and "wf_kv_dequant" in fake.calls
+    for name in ("wf_kv_append_fp8_chunks", "wf_kv_dequant_chunks", "wf_kv_append_publish_fp8",
+                 "wf_kv_dequant_published"):
+        assert name in fake.calls
 
 
 @pytest.mark.parametrize("case", [
     "k_rows", "v_shape", "k_heads", "pt_1d", "pt_width", "layer_out", "q_rows", "q_dim", "out",
     "lse_transposed", "row_short", "pool_mismatch", "fp8_scale", "dequant_geometry",
-    "flags_small", "flags_row_small",
+    "flags_small", "flags_row_small", "range_rows", "range_dequant_geometry",
+    "fp8_publish_rows", "fp8_publish_flags_small", "fp8_dequant_flags_row_small",
 ])
 def test_malformed_arguments_raise_before_any_launch(fake, case):
     lay = _layer()
@@ -133,6 +145,18 @@ def test_malformed_arguments_raise_before_any_launch(fake, case):
                                                       pt, lay.desc, 1),
         "flags_row_small": lambda: _abi.attn_forward_published(
             q, lay.pool.k, lay.pool.v, row, lay.desc, 0.1, out, flags[0, :2].contiguous(), 1),
+        # chunks [1, 3) hold 90 rows, not 130
+        "range_rows": lambda: _abi.kv_append_fp8_chunks(*fp.tensors, 0, 1, 3, _kv(130), _kv(130),
+                                                        pt, lay.desc),
+        "range_dequant_geometry": lambda: _abi.kv_dequant_chunks(
+            *fp.tensors, lay.pool.k[:9].contiguous(), lay.pool.v[:9].contiguous(), 0, 0, 3, pt,
+            lay.desc),
+        "fp8_publish_rows": lambda: _abi.kv_append_publish_fp8(*fp.tensors, flags, [], 0, 1,
+                                                               _kv(40), _kv(40), pt, lay.desc, 1),
+        "fp8_publish_flags_small": lambda: _abi.kv_append_publish_fp8(
+            *fp.tensors, flags[:, :2].contiguous(), [], 0, 0, k, v, pt, lay.desc, 1),
+        "fp8_dequant_flags_row_small": lambda: _abi.kv_dequant_published(
+            *fp.tensors, lay.pool.k, lay.pool.v, 0, 0, pt, lay.desc, flags[0, :2].contiguous(), 1),
     }
     with pytest.raises(ValueError):
         calls[case]()
