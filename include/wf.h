@@ -421,7 +421,9 @@ int wf_qk_quantize_i8(const void* q, const wf_kv_pool_t* kv_pages, const int32_t
 
 /* wf_attn_forward on quantized Q and K (filled by wf_qk_quantize_i8 for the same wavefront and
  * page table); V is read from kv_pages as in wf_attn_forward.  out, lse_or_null and errors as
- * wf_attn_forward.  Asynchronous on `stream`. */
+ * wf_attn_forward; WF_ERR_INVALID_ARG for a null field of qk or unaligned codes.  The call reads
+ * q_scale and k_scale as fp32 arrays: pass the struct the quantize call accepted (which checked
+ * their 4-byte alignment) -- this call does not check it again.  Asynchronous on `stream`. */
 int wf_attn_forward_i8(const wf_qk_i8_t* qk, const wf_kv_pool_t* kv_pages,
                        const int32_t* page_table_row, const wf_wavefront_t* wf, float scale,
                        void* out, float* lse_or_null, wf_stream_t stream);
@@ -459,7 +461,8 @@ int wf_qk_quantize_e4m3(const void* q, const wf_kv_pool_t* kv_pages,
                         const wf_qk_e4m3_t* qk, wf_stream_t stream);
 
 /* wf_attn_forward on e4m3 Q and K (filled by wf_qk_quantize_e4m3 for the same wavefront and page
- * table); V is read from kv_pages.  out, lse_or_null and errors as wf_attn_forward. */
+ * table); V is read from kv_pages.  out, lse_or_null and errors as wf_attn_forward_i8, and the
+ * same rule for the scales: pass the struct the quantize call accepted. */
 int wf_attn_forward_e4m3(const wf_qk_e4m3_t* qk, const wf_kv_pool_t* kv_pages,
                          const int32_t* page_table_row, const wf_wavefront_t* wf, float scale,
                          void* out, float* lse_or_null, wf_stream_t stream);

@@ -195,3 +195,76 @@ def test_fp8_validation_errors_without_a_gpu(abi):
     if not torch.cuda.is_available():
         assert append(_fp8_pool(abi)) == abi.WF_ERR_NO_DEVICE
         assert dequant(_fp8_pool(abi), _pool(abi)) == abi.WF_ERR_NO_DEVICE
+
+
+def _qk(abi, e4m3, **kw):
+    fields = abi.QK_E4M3_FIELDS if e4m3 else abi.QK_I8_FIELDS
+    args = {n: FAKE for n in fields}
+    args.update(kw)
+    return (abi.QkE4m3 if e4m3 else abi.QkI8)(**args)
+
+
+@pytest.mark.parametrize("e4m3", [False, True], ids=["int8", "e4m3"])
+def test_8bit_tier_validation_errors_without_a_gpu(abi, e4m3):
+    """The INT8 / FP8 attention tiers answer bad arguments, and empty work, before any device
+    work; a valid call on a machine without a GPU reports WF_ERR_NO_DEVICE."""
+    desc = abi.WavefrontDesc([0, 64, 128, 200], [0, 200, 1000], 1, 8)
+    empty = abi.WavefrontDesc([0, 64, 64], [0, 0], 1, 8)
+    tier = "e4m3" if e4m3 else "i8"
+    pt = ctypes.cast(ctypes.c_void_p(FAKE), ctypes.POINTER(ctypes.c_int32))
+
+    def quantize(qk, pool=None, wf=desc, q=FAKE):
+        return getattr(abi.lib, f"wf_qk_quantize_{tier}")(
+            q, ctypes.byref(pool or _pool(abi)), pt, ctypes.byref(wf.c),
+            ctypes.byref(qk) if qk is not None else None, None)
+
+    def forward(qk, pool=None, wf=desc):
+        return getattr(abi.lib, f"wf_attn_forward_{tier}")(
+            ctypes.byref(qk) if qk is not None else None, ctypes.byref(pool or _pool(abi)), pt,
+            ctypes.byref(wf.c), 0.1, FAKE, None, None)
+
+    ok = _qk(abi, e4m3)
+    assert quantize(None) == abi.WF_ERR_INVALID_ARG
+    assert quantize(ok, q=FAKE + 8) == abi.WF_ERR_INVALID_ARG                  # q unaligned
+    assert quantize(_qk(abi, e4m3, q_codes=FAKE + 8)) == abi.WF_ERR_INVALID_ARG
+    assert quantize(_qk(abi, e4m3, k_scale=FAKE + 2)) == abi.WF_ERR_INVALID_ARG
+    assert quantize(ok, pool=_pool(abi, head_dim=64)) == abi.WF_ERR_SHAPE
+    assert quantize(ok, wf=empty) == abi.WF_OK                                 # no query rows
+    assert forward(None) == abi.WF_ERR_INVALID_ARG
+    assert forward(_qk(abi, e4m3, k_codes=FAKE + 8)) == abi.WF_ERR_INVALID_ARG
+    assert forward(_qk(abi, e4m3, q_scale=None)) == abi.WF_ERR_INVALID_ARG
+    assert forward(_qk(abi, e4m3, q_codes=FAKE + 8)) == abi.WF_ERR_INVALID_ARG
+    assert forward(ok, pool=_pool(abi, head_dim=64)) == abi.WF_ERR_SHAPE
+    assert forward(ok, wf=empty) == abi.WF_OK
+    if not e4m3:
+        assert quantize(_qk(abi, e4m3, k_sum=FAKE + 4)) == abi.WF_ERR_INVALID_ARG  # fp64
+        assert quantize(_qk(abi, e4m3, k_mean=None)) == abi.WF_ERR_INVALID_ARG
+    if not torch.cuda.is_available():
+        assert quantize(ok) == abi.WF_ERR_NO_DEVICE
+        assert forward(ok) == abi.WF_ERR_NO_DEVICE
+
+
+def test_fp8_range_validation_errors_without_a_gpu(abi):
+    """The chunk-range forms of the FP8 append and conversion: the range [begin, end) must be
+    non-empty and inside the wavefront; empty chunks are no work."""
+    desc = abi.WavefrontDesc([0, 64, 128, 200], [0, 200, 1000], 1, 8)
+    pt = ctypes.cast(ctypes.c_void_p(FAKE), ctypes.POINTER(ctypes.c_int32))
+
+    def append(begin, end, k=FAKE, wf=desc):
+        return abi.lib.wf_kv_append_fp8_chunks(ctypes.byref(_fp8_pool(abi)), 0, begin, end, k,
+                                               FAKE, pt, ctypes.byref(wf.c), None)
+
+    def dequant(begin, end, dst=None):
+        return abi.lib.wf_kv_dequant_chunks(ctypes.byref(_fp8_pool(abi)),
+                                            ctypes.byref(dst or _pool(abi)), 0, begin, end, pt,
+                                            ctypes.byref(desc.c), None)
+    for begin, end in ((1, 1), (2, 1), (-1, 2), (0, 4)):
+        assert append(begin, end) == abi.WF_ERR_INVALID_ARG
+        assert dequant(begin, end) == abi.WF_ERR_INVALID_ARG
+    assert append(0, 3, k=FAKE + 2) == abi.WF_ERR_INVALID_ARG
+    assert dequant(0, 3, dst=_pool(abi, num_heads=3)) == abi.WF_ERR_SHAPE
+    empty = abi.WavefrontDesc([0, 64, 64, 64], [0, 0, 0], 1, 8)
+    assert append(1, 3, wf=empty) == abi.WF_OK                                  # no rows
+    if not torch.cuda.is_available():
+        assert append(0, 3) == abi.WF_ERR_NO_DEVICE
+        assert dequant(1, 3) == abi.WF_ERR_NO_DEVICE
