@@ -188,3 +188,36 @@ def test_tensors_of_one_allocation_are_mapped_once():
         assert peer_fp8 == (mapped + 768, mapped + 1024, mapped + 1280, mapped + 1536,
                             mapped + 512)                              # flags come last
         assert dests == [peer_fp8]
+
+
+def _mixed_fp8_worker(rank, world, port, results):
+    """Rank 0 passes an FP8 pool, rank 1 none: both ranks see every rank's handles after the one
+    exchange, so both refuse the same way and neither waits in a collective for the other."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        _fake_ipc(rank)
+        k, v = torch.zeros(64, dtype=torch.bfloat16), torch.zeros(64, dtype=torch.bfloat16)
+        flags = wave.new_flags(1, "cpu")
+        fp8 = [torch.zeros(64, dtype=torch.uint8) for _ in range(2)] + \
+            [torch.zeros(8, dtype=torch.float32) for _ in range(2)]
+        try:
+            wave.PublishedPools(k, v, flags, fp8=fp8 if rank == 0 else None)
+            results[rank] = "accepted"
+        except ValueError as e:
+            results[rank] = str(e)
+        dist.barrier()                      # both ranks still reach the next collective
+    finally:
+        dist.destroy_process_group()
+
+
+def test_an_fp8_pool_on_some_ranks_only_is_refused_everywhere():
+    world, port = 2, _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        results = m.dict()
+        mp.start_processes(_mixed_fp8_worker, args=(world, port, results), nprocs=world,
+                           start_method="spawn", join=True)
+        res = dict(results)
+    assert set(res) == {0, 1}
+    assert all("FP8 pool" in msg for msg in res.values()), res
